@@ -1,0 +1,686 @@
+// pod_attn_api.cpp -- C ABI, argument validation and the host planner of
+// libpod_attn.so. See include/pod_attn.h for the contract.
+//
+// Planner (POD-Attention §4.2.2-§4.2.3 and §5.4): splits the hybrid batch into
+// prefill units (request, head, 128-row query tile, KV split) and decode units
+// (request, KV head, KV split). Prefill KV splits are capped so the prefill
+// units stay within two waves of persistent slots (§4.2.3); the per-SM claim
+// ratio is proportional to the two queues' lengths (§5.4.2). The plan is a
+// pure function of the shapes and the SM count, so FUSED, SERIAL and
+// TWO_STREAM compute bitwise-identical results.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "pod_attn.h"
+#include "pod_plan.h"
+
+namespace pod {
+cudaError_t kernels_init(int D);
+int fused_smem_bytes(int D);
+int decode_smem_bytes(int D);
+cudaError_t launch_fused(const Plan& P, const TmaDescs& T, int grid, int allow_prefill,
+                         int allow_decode, cudaStream_t s);
+cudaError_t launch_decode(const Plan& P, cudaStream_t s);
+cudaError_t launch_merge(const Plan& P, cudaStream_t s);
+}  // namespace pod
+
+using namespace pod;
+
+namespace {
+
+constexpr int kRing = 8;            // pinned host plan slots
+constexpr int kMaxPrefillSplit = 16;
+constexpr int kDecSplitMin = 512;   // keys per decode split, smallest
+constexpr int kDecSplitMax = 1 << 20;
+constexpr int kStatsInts = kMaxSmid * 2;
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct DeviceGuard {
+  int prev = -1;
+  bool ok = false;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) != cudaSuccess) return;
+    ok = (prev == dev) || (cudaSetDevice(dev) == cudaSuccess);
+  }
+  ~DeviceGuard() {
+    int cur = -1;
+    if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+  }
+};
+
+// Byte offsets of one plan inside the plan buffer (host slot and device copy
+// have the same layout). Everything before `tables` is zeroed each call.
+struct PlanLayout {
+  size_t ctl, ticket, stats, pgroup, dgroup, tables, preq, punits, dreq, dunit, end;
+};
+
+}  // namespace
+
+struct pod_attn_ctx {
+  pod_attn_config cfg{};
+  int device = 0, num_sms = 0, slots_per_sm = kFusedSlotsPerSm;
+  int H = 0, Hk = 0, G = 0, D = 0;
+  int cap_punits = 0, cap_pgroups = 0, cap_pslots = 0;
+  int cap_dunits = 0, cap_dgroups = 0, cap_dslots = 0, cap_dreqs = 0;
+  size_t plan_cap = 0;
+  char* d_plan = nullptr;
+  float* d_ppart_o = nullptr;
+  float* d_ppart_lse = nullptr;
+  float* d_dpart_o = nullptr;
+  float* d_dpart_lse = nullptr;
+  int* d_misc = nullptr;  // [0] status, [1] never-set flag
+  char* h_plan[kRing] = {};
+  cudaEvent_t h_ev[kRing] = {};
+  int ring_i = 0;
+  cudaStream_t side = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+  PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  pod_plan_info last{};
+  PlanLayout lay{};
+  // scratch for the planner (reused, sized at create)
+  std::vector<PrefillUnit> units_tmp;
+  std::vector<int> units_key;
+};
+
+namespace {
+
+PlanLayout plan_layout(const pod_attn_ctx* c) {
+  PlanLayout L{};
+  size_t o = 0;
+  L.ctl = o; o += 64;
+  L.ticket = o; o += sizeof(int) * kMaxSmid;
+  L.stats = o; o += sizeof(int) * kStatsInts;
+  L.pgroup = o; o = align_up(o + sizeof(int) * (size_t)c->cap_pgroups, 64);
+  L.dgroup = o; o = align_up(o + sizeof(int) * (size_t)c->cap_dgroups, 64);
+  L.tables = o;
+  L.preq = o; o = align_up(o + sizeof(PrefillReq) * kMaxPrefillReqs, 64);
+  L.punits = o; o = align_up(o + sizeof(PrefillUnit) * (size_t)c->cap_punits, 64);
+  L.dreq = o; o = align_up(o + sizeof(DecodeReq) * (size_t)c->cap_dreqs, 64);
+  L.dunit = o; o = align_up(o + sizeof(int) * (size_t)c->cap_dunits, 64);
+  L.end = o;
+  return L;
+}
+
+int cuda_fail() { return POD_ECUDA; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int make_map(pod_attn_ctx* c, CUtensorMap* m, const void* base, uint64_t heads, uint64_t rows,
+             uint32_t box_rows) {
+  const uint64_t D = (uint64_t)c->D;
+  cuuint64_t dims[3] = {D, heads, rows};
+  cuuint64_t strides[2] = {D * 2, heads * D * 2};
+  cuuint32_t box[3] = {64, 1, box_rows};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = c->encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? POD_OK : POD_ECUDA;
+}
+
+// ----------------------------------------------------------------- validation
+int check_prefill(const pod_attn_ctx* c, const pod_prefill_args* a, long long* total_tokens) {
+  *total_tokens = 0;
+  if (!a || a->num_reqs == 0) return POD_OK;
+  if (a->num_reqs < 0) return POD_EINVAL;
+  if (a->num_reqs > c->cfg.max_prefill_reqs || a->num_reqs > kMaxPrefillReqs) return POD_ECAPACITY;
+  if (!a->chunk_lens || !a->prior_lens) return POD_EINVAL;
+  long long tot = 0;
+  for (int i = 0; i < a->num_reqs; ++i) {
+    const long long cl = a->chunk_lens[i], pl = a->prior_lens[i];
+    if (cl < 0 || pl < 0) return POD_EINVAL;
+    if (cl > 0 && cl + pl > c->cfg.max_kv_tokens) return POD_ECAPACITY;
+    if (cl + pl > (1LL << 30)) return POD_ECAPACITY;
+    tot += cl;
+  }
+  if (tot > c->cfg.max_prefill_tokens) return POD_ECAPACITY;
+  *total_tokens = tot;
+  if (tot == 0) return POD_OK;
+  if (!a->q || !a->o || !a->lse) return POD_EINVAL;
+  if (!aligned16(a->q) || !aligned16(a->o) || (reinterpret_cast<uintptr_t>(a->lse) & 3u))
+    return POD_EINVAL;
+  if (c->cfg.kv_layout == POD_KV_CONTIGUOUS) {
+    if (!a->k_ptrs || !a->v_ptrs) return POD_EINVAL;
+    for (int i = 0; i < a->num_reqs; ++i) {
+      if (a->chunk_lens[i] == 0) continue;
+      if (!a->k_ptrs[i] || !a->v_ptrs[i]) return POD_EINVAL;
+      if (!aligned16(a->k_ptrs[i]) || !aligned16(a->v_ptrs[i])) return POD_EINVAL;
+    }
+  } else {
+    if (!a->k_pool || !a->v_pool || !a->block_table || a->pool_blocks <= 0) return POD_EINVAL;
+    if (!aligned16(a->k_pool) || !aligned16(a->v_pool)) return POD_EINVAL;
+    if (a->pool_blocks * 16 > (1LL << 31)) return POD_ECAPACITY;
+    for (int i = 0; i < a->num_reqs; ++i) {
+      if (a->chunk_lens[i] == 0) continue;
+      const long long need = (a->chunk_lens[i] + (long long)a->prior_lens[i] + 15) / 16;
+      if (a->block_table_stride < need) return POD_EINVAL;
+    }
+  }
+  return POD_OK;
+}
+
+int check_decode(const pod_attn_ctx* c, const pod_decode_args* a) {
+  if (!a || a->num_reqs == 0) return POD_OK;
+  if (a->num_reqs < 0) return POD_EINVAL;
+  if (a->num_reqs > c->cfg.max_decode_reqs || a->num_reqs > c->cap_dreqs) return POD_ECAPACITY;
+  if (!a->ctx_lens || !a->q || !a->o || !a->lse) return POD_EINVAL;
+  if (!aligned16(a->q) || !aligned16(a->o) || (reinterpret_cast<uintptr_t>(a->lse) & 3u))
+    return POD_EINVAL;
+  for (int i = 0; i < a->num_reqs; ++i) {
+    if (a->ctx_lens[i] < 1) return POD_EINVAL;
+    if (a->ctx_lens[i] > c->cfg.max_kv_tokens) return POD_ECAPACITY;
+  }
+  if (c->cfg.kv_layout == POD_KV_CONTIGUOUS) {
+    if (!a->k_ptrs || !a->v_ptrs) return POD_EINVAL;
+    for (int i = 0; i < a->num_reqs; ++i) {
+      if (!a->k_ptrs[i] || !a->v_ptrs[i]) return POD_EINVAL;
+      if (!aligned16(a->k_ptrs[i]) || !aligned16(a->v_ptrs[i])) return POD_EINVAL;
+    }
+  } else {
+    if (!a->k_pool || !a->v_pool || !a->block_table || a->pool_blocks <= 0) return POD_EINVAL;
+    if (!aligned16(a->k_pool) || !aligned16(a->v_pool)) return POD_EINVAL;
+    for (int i = 0; i < a->num_reqs; ++i)
+      if (a->block_table_stride < (a->ctx_lens[i] + 15) / 16) return POD_EINVAL;
+  }
+  return POD_OK;
+}
+
+// ----------------------------------------------------------------- planner
+// Fills the host slot `h` and the kernel parameters. Returns a pod_status.
+int build_plan(pod_attn_ctx* c, const pod_prefill_args* pa, const pod_decode_args* da, char* h,
+               Plan* P, TmaDescs* T, size_t* copy_bytes) {
+  const PlanLayout& L = c->lay;
+  std::memset(h, 0, L.tables);
+  const int H = c->H, Hk = c->Hk;
+  const int np = (pa ? pa->num_reqs : 0);
+  const int nd = (da ? da->num_reqs : 0);
+  const bool paged = c->cfg.kv_layout == POD_KV_PAGED;
+  const int slots = c->num_sms * c->slots_per_sm;
+
+  // ---- prefill
+  PrefillReq* preq = reinterpret_cast<PrefillReq*>(h + L.preq);
+  PrefillUnit* punits = reinterpret_cast<PrefillUnit*>(h + L.punits);
+  long long tiles = 0;
+  for (int p = 0; p < np; ++p) tiles += (long long)((pa->chunk_lens[p] + kQTile - 1) / kQTile) * H;
+  int split_base = 1;
+  if (tiles > 0 && tiles < 2LL * slots) split_base = (int)std::max(1LL, (2LL * slots) / tiles);
+  int n_pu = 0, n_pg = 0, n_ps = 0, max_split = 1, q_row = 0;
+  c->units_tmp.clear();
+  c->units_key.clear();
+  for (int p = 0; p < np; ++p) {
+    PrefillReq& R = preq[p];
+    const int chunk = pa->chunk_lens[p], prior = pa->prior_lens[p];
+    R.prior = prior;
+    R.chunk = chunk;
+    R.q_row0 = q_row;
+    R.n_qtiles = (chunk + kQTile - 1) / kQTile;
+    R.kv_len = prior + chunk;
+    R.bt_row = p;
+    q_row += chunk;
+    if (chunk == 0) {
+      R.n_split = 1;
+      continue;
+    }
+    // smallest tile's KV range, in 64-key tiles; keep >= 4 tiles per split
+    const int min_tiles = (prior + std::min(chunk, kQTile) + kKVTile - 1) / kKVTile;
+    int split = std::min(split_base, std::max(1, min_tiles / 4));
+    split = std::min(split, kMaxPrefillSplit);
+    R.n_split = split;
+    R.n_kvtiles_max = (prior + chunk + kKVTile - 1) / kKVTile;
+    if (split > 1) {
+      R.group0 = n_pg;
+      R.slot0 = n_ps;
+      n_pg += R.n_qtiles * H;
+      n_ps += R.n_qtiles * H * split;
+    }
+    max_split = std::max(max_split, split);
+    for (int qt = 0; qt < R.n_qtiles; ++qt) {
+      const int kv_hi = prior + std::min(chunk, (qt + 1) * kQTile);
+      const int work = (kv_hi + kKVTile - 1) / kKVTile / split;
+      for (int hh = 0; hh < H; ++hh)
+        for (int sp = 0; sp < split; ++sp) {
+          c->units_tmp.push_back(PrefillUnit{p, hh, qt, sp});
+          c->units_key.push_back(work);
+        }
+    }
+  }
+  n_pu = (int)c->units_tmp.size();
+  if (n_pu > c->cap_punits || n_pg > c->cap_pgroups || n_ps > c->cap_pslots) return POD_ECAPACITY;
+  {
+    // longest units first (LPT) so the tail of the queue is short work
+    std::vector<int> idx(n_pu);
+    for (int i = 0; i < n_pu; ++i) idx[i] = i;
+    std::stable_sort(idx.begin(), idx.end(),
+                     [&](int a, int b) { return c->units_key[a] > c->units_key[b]; });
+    for (int i = 0; i < n_pu; ++i) punits[i] = c->units_tmp[idx[i]];
+  }
+
+  // ---- decode
+  DecodeReq* dreq = reinterpret_cast<DecodeReq*>(h + L.dreq);
+  int* dunit = reinterpret_cast<int*>(h + L.dunit);
+  long long key_heads = 0;
+  for (int r = 0; r < nd; ++r) key_heads += (long long)da->ctx_lens[r] * Hk;
+  // enough units to keep every decode warp busy several times over
+  const long long target = 8LL * c->num_sms * 8;
+  int split_len = kDecSplitMin;
+  auto count_units = [&](int sl) {
+    long long n = 0;
+    for (int r = 0; r < nd; ++r) n += (long long)((da->ctx_lens[r] + sl - 1) / sl) * Hk;
+    return n;
+  };
+  while (split_len < kDecSplitMax && count_units(split_len) > std::max(target, (long long)nd * Hk))
+    split_len *= 2;
+  while (split_len < kDecSplitMax && count_units(split_len) > c->cap_dunits) split_len *= 2;
+  (void)key_heads;
+  int n_du = 0, n_dg = 0, n_ds = 0;
+  for (int r = 0; r < nd; ++r) {
+    DecodeReq& R = dreq[r];
+    const int len = da->ctx_lens[r];
+    R.k = paged ? nullptr : static_cast<const uint16_t*>(da->k_ptrs[r]);
+    R.v = paged ? nullptr : static_cast<const uint16_t*>(da->v_ptrs[r]);
+    R.len = len;
+    R.n_split = (len + split_len - 1) / split_len;
+    R.unit0 = n_du;
+    R.bt_row = r;
+    if (R.n_split > 1) {
+      R.group0 = n_dg;
+      R.slot0 = n_ds;
+      n_dg += Hk;
+      n_ds += R.n_split * Hk;
+    }
+    const int nu = R.n_split * Hk;
+    if (n_du + nu > c->cap_dunits) return POD_ECAPACITY;
+    for (int i = 0; i < nu; ++i) dunit[n_du + i] = r;
+    n_du += nu;
+  }
+  if (n_dg > c->cap_dgroups || n_ds > c->cap_dslots) return POD_ECAPACITY;
+
+  // ---- claim ratio (per-SM Bresenham over tickets): prefill share of claims
+  const long long dclaims = (n_du + kFusedWarps - 1) / kFusedWarps;
+  int rho_num = n_pu, rho_den = n_pu + (int)dclaims;
+  if (rho_den == 0) rho_den = 1;
+
+  // ---- kernel parameters
+  Plan& Q = *P;
+  std::memset(&Q, 0, sizeof(Q));
+  Q.H = H;
+  Q.Hk = Hk;
+  Q.G = c->G;
+  Q.D = c->D;
+  Q.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)c->D));
+  Q.n_prefill_units = n_pu;
+  Q.n_decode_units = n_du;
+  Q.n_prefill_reqs = np;
+  Q.n_decode_reqs = nd;
+  Q.dec_split_len = split_len;
+  Q.rho_num = rho_num;
+  Q.rho_den = rho_den;
+  Q.paged = paged ? 1 : 0;
+  Q.bt_stride_p = (np && paged) ? pa->block_table_stride : 0;
+  Q.bt_stride_d = (nd && paged) ? da->block_table_stride : 0;
+  Q.flags = (int)c->cfg.flags;
+  Q.wait_budget = kDefaultWaitBudget;
+  char* dp = c->d_plan;
+  Q.preq = reinterpret_cast<const PrefillReq*>(dp + L.preq);
+  Q.punits = reinterpret_cast<const PrefillUnit*>(dp + L.punits);
+  Q.dreq = reinterpret_cast<const DecodeReq*>(dp + L.dreq);
+  Q.dunit_req = reinterpret_cast<const int*>(dp + L.dunit);
+  if (np) {
+    Q.q_p = static_cast<const uint16_t*>(pa->q);
+    Q.o_p = static_cast<uint16_t*>(pa->o);
+    Q.lse_p = pa->lse;
+    Q.bt_p = paged ? pa->block_table : nullptr;
+  }
+  if (nd) {
+    Q.q_d = static_cast<const uint16_t*>(da->q);
+    Q.o_d = static_cast<uint16_t*>(da->o);
+    Q.lse_d = da->lse;
+    Q.bt_d = paged ? da->block_table : nullptr;
+  }
+  if (paged) {
+    Q.k_pool = static_cast<const uint16_t*>(nd ? da->k_pool : (np ? pa->k_pool : nullptr));
+    Q.v_pool = static_cast<const uint16_t*>(nd ? da->v_pool : (np ? pa->v_pool : nullptr));
+    Q.pool_blocks = (int)std::min<long long>(nd ? da->pool_blocks : (np ? pa->pool_blocks : 0),
+                                             1LL << 30);
+  }
+  Q.ppart_o = c->d_ppart_o;
+  Q.ppart_lse = c->d_ppart_lse;
+  Q.dpart_o = c->d_dpart_o;
+  Q.dpart_lse = c->d_dpart_lse;
+  Q.ctl = reinterpret_cast<int*>(dp + L.ctl);
+  Q.sm_ticket = reinterpret_cast<int*>(dp + L.ticket);
+  Q.stats = reinterpret_cast<int*>(dp + L.stats);
+  Q.pgroup_ctr = reinterpret_cast<int*>(dp + L.pgroup);
+  Q.dgroup_ctr = reinterpret_cast<int*>(dp + L.dgroup);
+  Q.status = c->d_misc;
+  Q.never_set = c->d_misc + 1;
+
+  // ---- TMA descriptors (prefill only)
+  std::memset(T, 0, sizeof(*T));
+  if (n_pu > 0) {
+    const long long tp = q_row;
+    int rc = make_map(c, &T->q, pa->q, (uint64_t)H, (uint64_t)tp, kQTile);
+    if (rc) return rc;
+    if (!paged) {
+      for (int p = 0; p < np; ++p) {
+        if (pa->chunk_lens[p] == 0) continue;
+        const uint64_t len = (uint64_t)pa->chunk_lens[p] + (uint64_t)pa->prior_lens[p];
+        rc = make_map(c, &T->k[p], pa->k_ptrs[p], (uint64_t)Hk, len, kKVTile);
+        if (rc) return rc;
+        rc = make_map(c, &T->v[p], pa->v_ptrs[p], (uint64_t)Hk, len, kKVTile);
+        if (rc) return rc;
+      }
+    } else {
+      const uint64_t rows = (uint64_t)pa->pool_blocks * 16;
+      rc = make_map(c, &T->k[0], pa->k_pool, (uint64_t)Hk, rows, 16);
+      if (rc) return rc;
+      rc = make_map(c, &T->v[0], pa->v_pool, (uint64_t)Hk, rows, 16);
+      if (rc) return rc;
+    }
+  }
+  // ---- record
+  c->last.num_sms = c->num_sms;
+  c->last.slots_per_sm = c->slots_per_sm;
+  c->last.prefill_units = n_pu;
+  c->last.prefill_split = np ? max_split : 0;
+  c->last.decode_units = n_du;
+  c->last.decode_split_len = nd ? split_len : 0;
+  c->last.ratio_num = rho_num;
+  c->last.ratio_den = rho_den;
+  size_t used = L.dunit + sizeof(int) * (size_t)n_du;
+  if (n_du == 0) used = L.dreq + sizeof(DecodeReq) * (size_t)nd;
+  if (nd == 0 && n_du == 0) used = L.punits + sizeof(PrefillUnit) * (size_t)n_pu;
+  *copy_bytes = std::max(used, L.tables);
+  c->last.plan_bytes = (long long)*copy_bytes;
+  return POD_OK;
+}
+
+int fused_grid(const pod_attn_ctx* c, const Plan& P, bool allow_decode) {
+  long long claims = P.n_prefill_units;
+  if (allow_decode) claims += (P.n_decode_units + kFusedWarps - 1) / kFusedWarps;
+  long long g = std::min<long long>((long long)c->num_sms * c->slots_per_sm, claims);
+  return (int)std::max<long long>(g, 1);
+}
+
+// Common front half of every call: pick a ring slot, plan, copy the plan.
+int stage_plan(pod_attn_ctx* c, const pod_prefill_args* pa, const pod_decode_args* da,
+               cudaStream_t s, Plan* P, TmaDescs* T) {
+  const int slot = c->ring_i;
+  c->ring_i = (c->ring_i + 1) % kRing;
+  if (cudaEventSynchronize(c->h_ev[slot]) != cudaSuccess) return POD_ECUDA;
+  size_t bytes = 0;
+  int rc = build_plan(c, pa, da, c->h_plan[slot], P, T, &bytes);
+  if (rc) return rc;
+  if (cudaMemcpyAsync(c->d_plan, c->h_plan[slot], bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return POD_ECUDA;
+  if (cudaEventRecord(c->h_ev[slot], s) != cudaSuccess) return POD_ECUDA;
+  return POD_OK;
+}
+
+}  // namespace
+
+// =================================================================== C ABI
+extern "C" {
+
+const char* pod_attn_strerror(int st) {
+  switch (st) {
+    case POD_OK: return "ok";
+    case POD_EINVAL: return "invalid argument";
+    case POD_EUNSUPPORTED: return "unsupported shape or layout";
+    case POD_ENOMEM: return "out of memory";
+    case POD_ECUDA: return "CUDA error";
+    case POD_ETIMEOUT: return "device wait timed out";
+    case POD_ECAPACITY: return "size exceeds the context's capacity";
+    default: return "unknown status";
+  }
+}
+
+int pod_attn_create(pod_attn_ctx** out, const pod_attn_config* cfg) {
+  if (!out || !cfg) return POD_EINVAL;
+  *out = nullptr;
+  const int H = cfg->num_qo_heads, Hk = cfg->num_kv_heads, D = cfg->head_dim;
+  if (H <= 0 || Hk <= 0 || H % Hk != 0) return POD_EINVAL;
+  if (cfg->max_prefill_reqs < 0 || cfg->max_prefill_tokens < 0 || cfg->max_decode_reqs < 0 ||
+      cfg->max_kv_tokens < 1)
+    return POD_EINVAL;
+  if (cfg->kv_layout != POD_KV_CONTIGUOUS && cfg->kv_layout != POD_KV_PAGED) return POD_EINVAL;
+  if (D != 64 && D != 128) return POD_EUNSUPPORTED;
+  if (H / Hk > kMaxGroup) return POD_EUNSUPPORTED;
+  if (cfg->kv_layout == POD_KV_PAGED && cfg->page_size != 16) return POD_EUNSUPPORTED;
+  if (cfg->max_prefill_reqs > kMaxPrefillReqs) return POD_ECAPACITY;
+  if (cfg->max_kv_tokens > (1LL << 30)) return POD_ECAPACITY;
+
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess) return POD_ECUDA;
+  if (cfg->device < 0 || cfg->device >= ndev) return POD_EINVAL;
+  DeviceGuard guard(cfg->device);
+  if (!guard.ok) return POD_ECUDA;
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, cfg->device) != cudaSuccess) return POD_ECUDA;
+  if (prop.major != 10 || prop.minor != 0) return POD_EUNSUPPORTED;  // built for sm_100a only
+
+  pod_attn_ctx* c = new (std::nothrow) pod_attn_ctx();
+  if (!c) return POD_ENOMEM;
+  c->cfg = *cfg;
+  c->device = cfg->device;
+  c->num_sms = prop.multiProcessorCount;
+  c->H = H;
+  c->Hk = Hk;
+  c->G = H / Hk;
+  c->D = D;
+
+  auto fail = [&](int code) {
+    pod_attn_destroy(c);
+    return code;
+  };
+  if (kernels_init(D) != cudaSuccess) return fail(POD_ECUDA);
+
+  // capacities
+  const int slots = c->num_sms * c->slots_per_sm;
+  const long long qtiles = (long long)cfg->max_prefill_tokens / kQTile + cfg->max_prefill_reqs;
+  c->cap_punits = (int)std::min<long long>(qtiles * H * kMaxPrefillSplit, 1 << 24);
+  c->cap_pgroups = (int)std::min<long long>(std::min<long long>(qtiles * H, 2LL * slots), 1 << 24);
+  c->cap_pslots = 2 * slots + kMaxPrefillSplit * H;  // split only when tiles < 2 waves
+  c->cap_pgroups = std::max(c->cap_pgroups, 1);
+  c->cap_dreqs = std::max(cfg->max_decode_reqs, 1);
+  c->cap_dunits = (int)std::max<long long>(16LL * c->num_sms * 8, (long long)c->cap_dreqs * Hk * 2);
+  c->cap_dgroups = c->cap_dreqs * Hk;
+  c->cap_dslots = c->cap_dunits;
+  c->lay = plan_layout(c);
+  c->plan_cap = c->lay.end;
+
+  if (cudaMalloc(&c->d_plan, c->plan_cap) != cudaSuccess) return fail(POD_ENOMEM);
+  if (cudaMalloc(&c->d_ppart_o, sizeof(float) * (size_t)c->cap_pslots * kQTile * D) != cudaSuccess)
+    return fail(POD_ENOMEM);
+  if (cudaMalloc(&c->d_ppart_lse, sizeof(float) * (size_t)c->cap_pslots * kQTile) != cudaSuccess)
+    return fail(POD_ENOMEM);
+  if (cudaMalloc(&c->d_dpart_o, sizeof(float) * (size_t)c->cap_dslots * kMaxGroup * D) !=
+      cudaSuccess)
+    return fail(POD_ENOMEM);
+  if (cudaMalloc(&c->d_dpart_lse, sizeof(float) * (size_t)c->cap_dslots * kMaxGroup) != cudaSuccess)
+    return fail(POD_ENOMEM);
+  if (cudaMalloc(&c->d_misc, 64) != cudaSuccess) return fail(POD_ENOMEM);
+  if (cudaMemset(c->d_misc, 0, 64) != cudaSuccess) return fail(POD_ECUDA);
+  if (cudaMemset(c->d_plan, 0, c->plan_cap) != cudaSuccess) return fail(POD_ECUDA);
+  for (int i = 0; i < kRing; ++i) {
+    if (cudaHostAlloc(reinterpret_cast<void**>(&c->h_plan[i]), c->plan_cap,
+                      cudaHostAllocDefault) != cudaSuccess)
+      return fail(POD_ENOMEM);
+    std::memset(c->h_plan[i], 0, c->plan_cap);
+    if (cudaEventCreateWithFlags(&c->h_ev[i], cudaEventDisableTiming) != cudaSuccess)
+      return fail(POD_ECUDA);
+  }
+  if (cudaStreamCreateWithFlags(&c->side, cudaStreamNonBlocking) != cudaSuccess)
+    return fail(POD_ECUDA);
+  if (cudaEventCreateWithFlags(&c->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&c->ev_join, cudaEventDisableTiming) != cudaSuccess)
+    return fail(POD_ECUDA);
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                       &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || !fn)
+    return fail(POD_ECUDA);
+  c->encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  c->units_tmp.reserve(1024);
+  c->units_key.reserve(1024);
+  if (cudaDeviceSynchronize() != cudaSuccess) return fail(POD_ECUDA);
+  *out = c;
+  return POD_OK;
+}
+
+int pod_attn_hybrid(pod_attn_ctx* c, const pod_prefill_args* pa, const pod_decode_args* da,
+                    int mode, void* stream) {
+  if (!c) return POD_EINVAL;
+  if (mode != POD_MODE_FUSED && mode != POD_MODE_SERIAL && mode != POD_MODE_TWO_STREAM)
+    return POD_EINVAL;
+  long long tp = 0;
+  int rc = check_prefill(c, pa, &tp);
+  if (rc) return rc;
+  rc = check_decode(c, da);
+  if (rc) return rc;
+  DeviceGuard guard(c->device);
+  if (!guard.ok) return POD_ECUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Plan P;
+  TmaDescs T;
+  rc = stage_plan(c, pa, da, s, &P, &T);
+  if (rc) return rc;
+  const bool has_p = P.n_prefill_units > 0, has_d = P.n_decode_units > 0;
+  if (!has_p && !has_d) return POD_OK;
+  if (mode == POD_MODE_FUSED) {
+    if (launch_fused(P, T, fused_grid(c, P, true), 1, 1, s) != cudaSuccess) return POD_ECUDA;
+    return POD_OK;
+  }
+  if (mode == POD_MODE_SERIAL) {
+    if (has_p && launch_fused(P, T, fused_grid(c, P, false), 1, 0, s) != cudaSuccess)
+      return POD_ECUDA;
+    if (has_d && (launch_decode(P, s) != cudaSuccess || launch_merge(P, s) != cudaSuccess))
+      return POD_ECUDA;
+    return POD_OK;
+  }
+  // TWO_STREAM
+  if (cudaEventRecord(c->ev_fork, s) != cudaSuccess) return POD_ECUDA;
+  if (cudaStreamWaitEvent(c->side, c->ev_fork, 0) != cudaSuccess) return POD_ECUDA;
+  if (has_p && launch_fused(P, T, fused_grid(c, P, false), 1, 0, s) != cudaSuccess)
+    return POD_ECUDA;
+  if (has_d && (launch_decode(P, c->side) != cudaSuccess || launch_merge(P, c->side) != cudaSuccess))
+    return POD_ECUDA;
+  if (cudaEventRecord(c->ev_join, c->side) != cudaSuccess) return POD_ECUDA;
+  if (cudaStreamWaitEvent(s, c->ev_join, 0) != cudaSuccess) return POD_ECUDA;
+  return POD_OK;
+}
+
+int pod_attn_prefill_only(pod_attn_ctx* c, const pod_prefill_args* pa, void* stream) {
+  if (!c) return POD_EINVAL;
+  long long tp = 0;
+  int rc = check_prefill(c, pa, &tp);
+  if (rc) return rc;
+  DeviceGuard guard(c->device);
+  if (!guard.ok) return POD_ECUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Plan P;
+  TmaDescs T;
+  rc = stage_plan(c, pa, nullptr, s, &P, &T);
+  if (rc) return rc;
+  if (P.n_prefill_units == 0) return POD_OK;
+  return launch_fused(P, T, fused_grid(c, P, false), 1, 0, s) == cudaSuccess ? POD_OK : POD_ECUDA;
+}
+
+int pod_attn_decode_only(pod_attn_ctx* c, const pod_decode_args* da, void* stream) {
+  if (!c) return POD_EINVAL;
+  int rc = check_decode(c, da);
+  if (rc) return rc;
+  DeviceGuard guard(c->device);
+  if (!guard.ok) return POD_ECUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Plan P;
+  TmaDescs T;
+  rc = stage_plan(c, nullptr, da, s, &P, &T);
+  if (rc) return rc;
+  if (P.n_decode_units == 0) return POD_OK;
+  if (launch_decode(P, s) != cudaSuccess || launch_merge(P, s) != cudaSuccess) return POD_ECUDA;
+  return POD_OK;
+}
+
+int pod_attn_status(pod_attn_ctx* c, void* stream) {
+  if (!c) return POD_EINVAL;
+  DeviceGuard guard(c->device);
+  if (!guard.ok) return POD_ECUDA;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return POD_ECUDA;
+  int st = 0;
+  if (cudaMemcpy(&st, c->d_misc, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return POD_ECUDA;
+  if (cudaMemset(c->d_misc, 0, sizeof(int)) != cudaSuccess) return POD_ECUDA;
+  return st;
+}
+
+int pod_attn_last_plan(const pod_attn_ctx* c, pod_plan_info* out) {
+  if (!c || !out) return POD_EINVAL;
+  *out = c->last;
+  return POD_OK;
+}
+
+int pod_attn_get_stats(pod_attn_ctx* c, void* stream, pod_stats* out) {
+  if (!c || !out) return POD_EINVAL;
+  if (!(c->cfg.flags & POD_FLAG_STATS)) return POD_EINVAL;
+  DeviceGuard guard(c->device);
+  if (!guard.ok) return POD_ECUDA;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return POD_ECUDA;
+  std::vector<int> st(kStatsInts);
+  if (cudaMemcpy(st.data(), c->d_plan + c->lay.stats, sizeof(int) * kStatsInts,
+                 cudaMemcpyDeviceToHost) != cudaSuccess)
+    return POD_ECUDA;
+  std::memset(out, 0, sizeof(*out));
+  out->num_sms = c->num_sms;
+  for (int i = 0; i < kMaxSmid; ++i) {
+    out->prefill_claims += st[2 * i];
+    out->decode_claims += st[2 * i + 1];
+    if (st[2 * i] > 0 && st[2 * i + 1] > 0) out->sms_with_both++;
+  }
+  return POD_OK;
+}
+
+int pod_attn_destroy(pod_attn_ctx* c) {
+  if (!c) return POD_OK;
+  int st = POD_OK;
+  {
+    DeviceGuard guard(c->device);
+    if (cudaDeviceSynchronize() != cudaSuccess) st = POD_ECUDA;
+    if (c->d_misc && st == POD_OK) {
+      int v = 0;
+      if (cudaMemcpy(&v, c->d_misc, sizeof(int), cudaMemcpyDeviceToHost) == cudaSuccess)
+        st = v;
+      else
+        st = POD_ECUDA;
+    }
+    cudaFree(c->d_plan);
+    cudaFree(c->d_ppart_o);
+    cudaFree(c->d_ppart_lse);
+    cudaFree(c->d_dpart_o);
+    cudaFree(c->d_dpart_lse);
+    cudaFree(c->d_misc);
+    for (int i = 0; i < kRing; ++i) {
+      if (c->h_plan[i]) cudaFreeHost(c->h_plan[i]);
+      if (c->h_ev[i]) cudaEventDestroy(c->h_ev[i]);
+    }
+    if (c->side) cudaStreamDestroy(c->side);
+    if (c->ev_fork) cudaEventDestroy(c->ev_fork);
+    if (c->ev_join) cudaEventDestroy(c->ev_join);
+  }
+  delete c;
+  return st;
+}
+
+}  // extern "C"

@@ -1,0 +1,945 @@
+// pod_kernels.cu -- sm_100a kernels of the hybrid prefill + decode attention.
+//
+// Roles (POD-Attention §4 "POD-Attention"; the paper's FlashAttention device
+// functions for A100 are prior art here, rebuilt for Blackwell):
+//  * prefill unit: one 128-row query tile of one head against a range of
+//    64-key KV tiles. A TMA producer warp stages Q and K/V (128-byte swizzle),
+//    one thread issues tcgen05.mma (S = Q K^T into TMEM, O += P V into TMEM),
+//    four softmax warps (one thread per query row = TMEM lane) run the online
+//    softmax and write P (bf16) into the K stage the S MMA just consumed.
+//  * decode unit: one warp (a "virtual decode CTA", paper §4.2.3) streams the
+//    K/V rows of (request, KV head, key split) with TMA bulk copies into a
+//    padded smem ring and runs S^T = K Q^T and O^T += V^T P^T on the legacy
+//    m16n8k16 tensor-core path with the G query heads of the group as N = 8
+//    (the paper's small decode tile, §4.2.1).
+//  * merge: log-sum-exp combination of split partials, in split order.
+//  * fused kernel: persistent CTAs (2 per SM) read %smid, take a ticket from
+//    that SM's counter and pick prefill or decode work in the planned ratio
+//    (§4.1 SM-aware scheduling, §4.4 persistent threads, §5.4.2 proportional
+//    allocation); the last CTA to finish a split group merges it, so no CTA
+//    ever waits for another (the digest's deadlock-free merge requirement).
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "pod_plan.h"
+#include "pod_ptx.cuh"
+
+namespace pod {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr int kStatusTimeout = -5;
+
+POD_DEV void set_status(const Plan& P, int code) { atomicCAS(P.status, 0, code); }
+
+// Bounded mbarrier wait. On timeout records POD_ETIMEOUT, raises the CTA's
+// abort flag and returns false; once the flag is up every later wait returns
+// false at once, so all roles reach the end of the CTA.
+POD_DEV bool wait_bar(uint32_t bar, uint32_t parity, const Plan& P, volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (clock64() - t0 > P.wait_budget) {
+      set_status(P, kStatusTimeout);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+// Warp-collective form: every lane gets the same answer, so warp-collective
+// instructions after it (tcgen05.ld, shuffles, ldmatrix) stay convergent.
+POD_DEV bool wait_bar_warp(uint32_t bar, uint32_t parity, const Plan& P,
+                           volatile int* abort_flag) {
+  const bool ok = wait_bar(bar, parity, P, abort_flag);
+  return __all_sync(0xffffffffu, ok);
+}
+// Drain wait used only after an abort: waits for an async copy or MMA this
+// thread issued itself, bounded, ignoring the abort flag.
+POD_DEV void drain_bar(uint32_t bar, uint32_t parity, long long budget) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > budget) return;
+  }
+}
+
+// ============================================================= smem layout
+template <int D>
+struct FusedLayout {
+  static constexpr int QB = kQTile * D * 2;   // Q tile bytes
+  static constexpr int KT = kKVTile * D * 2;  // one K (or V) tile
+  static constexpr int Q_OFF = 0;
+  static constexpr int K_OFF = Q_OFF + QB;
+  static constexpr int V_OFF = K_OFF + kPrefillStages * KT;
+  static constexpr int P_OFF = V_OFF + kPrefillStages * KT;  // own P buffer only when d < 128
+  static constexpr int P_BYTES = (D >= 128) ? 0 : kQTile * kKVTile * 2;
+  static constexpr int PREFILL_END = P_OFF + P_BYTES;
+  static constexpr int DEC_ROW = D * 2 + 16;  // padded row: conflict-free ldmatrix
+  static constexpr int DEC_STAGE = 2 * kDecTile * DEC_ROW;
+  static constexpr int DEC_WARP = kFusedDecStages * DEC_STAGE;
+  static constexpr int DEC_END = kFusedWarps * DEC_WARP;
+  static constexpr int DATA_END = PREFILL_END > DEC_END ? PREFILL_END : DEC_END;
+  static constexpr int BAR_OFF = (DATA_END + 127) & ~127;
+  // barrier indices
+  static constexpr int B_Q = 0;
+  static constexpr int B_KF = 1;
+  static constexpr int B_VF = B_KF + kPrefillStages;
+  static constexpr int B_KVE = B_VF + kPrefillStages;
+  static constexpr int B_SF = B_KVE + kPrefillStages;
+  static constexpr int B_SE = B_SF + 2;
+  static constexpr int B_PF = B_SE + 2;
+  static constexpr int B_PV = B_PF + 1;
+  static constexpr int B_DEC = B_PV + 1;
+  static constexpr int N_BARS = B_DEC + kFusedWarps * kFusedDecStages;
+  static constexpr int MISC_OFF = BAR_OFF + N_BARS * 8;
+  static constexpr int TOTAL = MISC_OFF + 64;
+  static constexpr int SMEM_BYTES = TOTAL + 1024;  // slack for 1024-byte alignment
+};
+
+template <int D>
+struct DecodeLayout {
+  static constexpr int ROW = D * 2 + 16;
+  static constexpr int STAGE = 2 * kDecTile * ROW;
+  static constexpr int WARP = kDecodeStages * STAGE;
+  static constexpr int BAR_OFF = kDecodeWarps * WARP;
+  static constexpr int SMEM_BYTES = BAR_OFF + kDecodeWarps * kDecodeStages * 8 + 16;
+};
+
+// ============================================================= LSE merge
+// One warp merges one output row of D values from n split partials, in split
+// order: M = max lse_s, w_s = exp(lse_s - M), O = sum w_s O_s / sum w_s,
+// LSE = M + ln sum w_s. Partials written by other CTAs are read with .cg.
+template <int D>
+POD_DEV void merge_row_warp(const float* po, long long po_stride, const float* pl,
+                            long long pl_stride, int n, uint16_t* out, float* lse_out, int lane) {
+  constexpr int PER = D / 32;
+  float M = -INFINITY;
+  for (int s = 0; s < n; ++s) M = fmaxf(M, __ldcg(pl + s * pl_stride));
+  float acc[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) acc[i] = 0.f;
+  float W = 0.f;
+  for (int s = 0; s < n; ++s) {
+    const float ls = __ldcg(pl + s * pl_stride);
+    const float w = (ls == -INFINITY) ? 0.f : ex2((ls - M) * kLog2e);
+    W += w;
+    const float* src = po + s * po_stride + lane * PER;
+    if constexpr (PER == 4) {
+      const float4 x = __ldcg(reinterpret_cast<const float4*>(src));
+      acc[0] = fmaf(w, x.x, acc[0]);
+      acc[1] = fmaf(w, x.y, acc[1]);
+      acc[2] = fmaf(w, x.z, acc[2]);
+      acc[3] = fmaf(w, x.w, acc[3]);
+    } else {
+      const float2 x = __ldcg(reinterpret_cast<const float2*>(src));
+      acc[0] = fmaf(w, x.x, acc[0]);
+      acc[1] = fmaf(w, x.y, acc[1]);
+    }
+  }
+  const float inv = 1.f / W;
+  if constexpr (PER == 4) {
+    uint2 v;
+    v.x = pack_bf16(acc[0] * inv, acc[1] * inv);
+    v.y = pack_bf16(acc[2] * inv, acc[3] * inv);
+    *reinterpret_cast<uint2*>(out + lane * 4) = v;
+  } else {
+    *reinterpret_cast<uint32_t*>(out + lane * 2) = pack_bf16(acc[0] * inv, acc[1] * inv);
+  }
+  if (lane == 0 && lse_out) *lse_out = M + logf(W);
+}
+
+// ============================================================= decode unit
+// One warp, one unit (request r, KV head g, keys [kbeg, kend)). The ring of
+// `NST` stages lives at `wsm` (each stage: 16 K rows then 16 V rows, padded);
+// `bar0` is the shared address of NST mbarriers. `ring` counts tiles this warp
+// has staged so far (carries the mbarrier phases across units).
+template <int D, int NST>
+POD_DEV bool decode_unit_warp(const Plan& P, int u, uint8_t* wsm, uint32_t bar0, uint32_t& ring,
+                              int lane, bool inline_merge, volatile int* abort_flag) {
+  constexpr int ROW = D * 2 + 16;
+  constexpr int STAGE = 2 * kDecTile * ROW;
+  constexpr int KS = D / 16;
+  const int r = P.dunit_req[u];
+  const DecodeReq R = P.dreq[r];
+  const int Hk = P.Hk, G = P.G;
+  const int local = u - R.unit0;
+  const int s = local / Hk;
+  const int g = local - s * Hk;
+  const int kbeg = s * P.dec_split_len;
+  const int kend = min(R.len, kbeg + P.dec_split_len);
+  const int n_tiles = (kend - kbeg + kDecTile - 1) / kDecTile;
+  const int q4 = lane & 3;
+  const int hrow = lane >> 2;  // query head within the group (B column / C row of S^T)
+
+  // Q^T as the B operand of S^T = K Q^T: lane holds Q[head lane/4][16kk + 2q4 (+1, +8, +9)].
+  uint32_t qb[KS][2];
+  {
+    const uint16_t* qrow = P.q_d + ((size_t)r * P.H + (size_t)g * G + hrow) * D;
+#pragma unroll
+    for (int kk = 0; kk < KS; ++kk) {
+      if (hrow < G) {
+        qb[kk][0] = __ldg(reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 2 * q4));
+        qb[kk][1] = __ldg(reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 2 * q4 + 8));
+      } else {
+        qb[kk][0] = 0u;
+        qb[kk][1] = 0u;
+      }
+    }
+  }
+  const size_t row_elems = (size_t)Hk * D;
+  auto row_off = [&](int key) -> size_t {
+    if (P.paged) {
+      int phys = __ldg(P.bt_d + (size_t)R.bt_row * P.bt_stride_d + (key >> 4));
+      phys = min(max(phys, 0), P.pool_blocks - 1);  // never read outside the pool
+      return ((size_t)phys * 16 + (key & 15)) * row_elems + (size_t)g * D;
+    }
+    return (size_t)key * row_elems + (size_t)g * D;
+  };
+  const uint16_t* kbase = P.paged ? P.k_pool : R.k;
+  const uint16_t* vbase = P.paged ? P.v_pool : R.v;
+  const uint32_t wsm_a = smem_u32(wsm);
+
+  auto issue = [&](int t) {
+    const uint32_t it = ring + t;
+    const uint32_t st = it % NST;
+    const uint32_t bar = bar0 + st * 8;
+    if (lane == 0) mbar_expect_tx(bar, 2 * kDecTile * D * 2);
+    __syncwarp();
+    int key = kbeg + t * kDecTile + (lane & 15);
+    key = min(key, kend - 1);  // ragged tail: re-read a valid row, masked below
+    const size_t off = row_off(key);
+    const uint16_t* src = (lane < 16) ? (kbase + off) : (vbase + off);
+    const uint32_t dst = wsm_a + st * STAGE + (lane < 16 ? 0 : kDecTile * ROW) + (lane & 15) * ROW;
+    bulk_load(dst, src, D * 2, bar);
+  };
+
+  fence_proxy_async_smem();
+  int issued = min(NST, n_tiles);  // tiles [0, issued) have been issued
+  for (int t = 0; t < issued; ++t) issue(t);
+
+  float o[KS][4];
+#pragma unroll
+  for (int mt = 0; mt < KS; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  const float sc = P.scale_log2;
+  bool ok = true;
+
+  for (int t = 0; t < n_tiles; ++t) {
+    const uint32_t it = ring + t;
+    const uint32_t st = it % NST;
+    if (!wait_bar_warp(bar0 + st * 8, (it / NST) & 1, P, abort_flag)) {
+      ok = false;
+      break;
+    }
+    const uint32_t kb = wsm_a + st * STAGE;
+    const uint32_t vb = kb + kDecTile * ROW;
+    // S^T[16 keys x 8 heads]
+    float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int kk = 0; kk < KS; ++kk) {
+      uint32_t a[4];
+      ldsm_x4(kb + (lane & 15) * ROW + (kk * 16 + 8 * (lane >> 4)) * 2, a);
+      mma_16816(c, a, qb[kk][0], qb[kk][1]);
+    }
+    const int key_a = kbeg + t * kDecTile + hrow;
+    float s0 = (key_a < kend) ? c[0] * sc : -INFINITY;
+    float s1 = (key_a < kend) ? c[1] * sc : -INFINITY;
+    float s2 = (key_a + 8 < kend) ? c[2] * sc : -INFINITY;
+    float s3 = (key_a + 8 < kend) ? c[3] * sc : -INFINITY;
+    float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+    }
+    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);  // finite: >= 1 valid key per tile
+    const float a0 = ex2(m0 - mn0), a1 = ex2(m1 - mn1);
+    m0 = mn0;
+    m1 = mn1;
+    const float p0 = ex2(s0 - mn0), p1 = ex2(s1 - mn1), p2 = ex2(s2 - mn0), p3 = ex2(s3 - mn1);
+    const uint32_t x01 = pack_bf16(p0, p1);  // key hrow
+    const uint32_t x23 = pack_bf16(p2, p3);  // key hrow + 8
+    // The normaliser sums the unrounded fp32 weights: summing the bf16-rounded
+    // ones would put their rounding (2^-9 relative) straight into the LSE.
+    l0 = l0 * a0 + (p0 + p2);
+    l1 = l1 * a1 + (p1 + p3);
+#pragma unroll
+    for (int mt = 0; mt < KS; ++mt) {
+      o[mt][0] *= a0;
+      o[mt][1] *= a1;
+      o[mt][2] *= a0;
+      o[mt][3] *= a1;
+    }
+    // P^T as the B operand: transpose each 8x8 (key x head) block.
+    const uint32_t b0 = movmatrix_t(x01);
+    const uint32_t b1 = movmatrix_t(x23);
+#pragma unroll
+    for (int mt = 0; mt < KS; ++mt) {
+      uint32_t a[4];
+      ldsm_x4_t(vb + ((lane & 7) + 8 * (lane >> 4)) * ROW + (mt * 16 + 8 * ((lane >> 3) & 1)) * 2,
+                a);
+      mma_16816(o[mt], a, b0, b1);
+    }
+    __syncwarp();
+    if (t + NST < n_tiles) {
+      fence_proxy_async_smem();
+      issue(t + NST);
+      issued = t + NST + 1;
+    }
+  }
+  if (!ok) {
+    // Abort: wait (bounded) for the copies this warp still has in flight --
+    // the last NST issued tiles -- so no copy lands after the CTA exits.
+    for (int t = max(0, issued - NST); t < issued; ++t) {
+      const uint32_t it = ring + t;
+      drain_bar(bar0 + (it % NST) * 8, (it / NST) & 1, P.wait_budget);
+    }
+    ring += n_tiles;
+    return false;
+  }
+  ring += n_tiles;
+
+  // l: sum of lane partials over the 8 lanes sharing q4.
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) {
+    l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+  }
+  const int h0 = 2 * q4, h1 = 2 * q4 + 1;  // heads of c0/c2 and c1/c3
+  if (R.n_split <= 1) {
+    const float i0 = 1.f / l0, i1 = 1.f / l1;
+    uint16_t* ob = P.o_d + ((size_t)r * P.H + (size_t)g * G) * D;
+#pragma unroll
+    for (int mt = 0; mt < KS; ++mt) {
+      const int d0 = mt * 16 + hrow;
+      if (h0 < G) {
+        ob[(size_t)h0 * D + d0] = (uint16_t)(pack_bf16(o[mt][0] * i0, 0.f) & 0xFFFF);
+        ob[(size_t)h0 * D + d0 + 8] = (uint16_t)(pack_bf16(o[mt][2] * i0, 0.f) & 0xFFFF);
+      }
+      if (h1 < G) {
+        ob[(size_t)h1 * D + d0] = (uint16_t)(pack_bf16(o[mt][1] * i1, 0.f) & 0xFFFF);
+        ob[(size_t)h1 * D + d0 + 8] = (uint16_t)(pack_bf16(o[mt][3] * i1, 0.f) & 0xFFFF);
+      }
+    }
+    if (hrow == 0) {
+      float* lb = P.lse_d + (size_t)r * P.H + (size_t)g * G;
+      if (h0 < G) lb[h0] = (m0 + log2f(l0)) * kLn2;
+      if (h1 < G) lb[h1] = (m1 + log2f(l1)) * kLn2;
+    }
+    return true;
+  }
+  // split: fp32 partial (normalised) + partial LSE
+  const int slot = R.slot0 + s * Hk + g;
+  float* po = P.dpart_o + (size_t)slot * kMaxGroup * D;
+  {
+    const float i0 = 1.f / l0, i1 = 1.f / l1;
+#pragma unroll
+    for (int mt = 0; mt < KS; ++mt) {
+      const int d0 = mt * 16 + hrow;
+      if (h0 < G) {
+        po[h0 * D + d0] = o[mt][0] * i0;
+        po[h0 * D + d0 + 8] = o[mt][2] * i0;
+      }
+      if (h1 < G) {
+        po[h1 * D + d0] = o[mt][1] * i1;
+        po[h1 * D + d0 + 8] = o[mt][3] * i1;
+      }
+    }
+    if (hrow == 0) {
+      float* pl = P.dpart_lse + (size_t)slot * kMaxGroup;
+      if (h0 < G) pl[h0] = (m0 + log2f(l0)) * kLn2;
+      if (h1 < G) pl[h1] = (m1 + log2f(l1)) * kLn2;
+    }
+  }
+  if (!inline_merge) return true;
+  __threadfence();
+  __syncwarp();
+  int last = 0;
+  if (lane == 0) last = (atomicAdd(P.dgroup_ctr + R.group0 + g, 1) == R.n_split - 1);
+  last = __shfl_sync(0xffffffffu, last, 0);
+  if (!last) return true;
+  __threadfence();
+  for (int i = 0; i < G; ++i) {
+    const int slot0 = R.slot0 + g;
+    merge_row_warp<D>(P.dpart_o + ((size_t)slot0 * kMaxGroup + i) * D, (long long)Hk * kMaxGroup * D,
+                      P.dpart_lse + (size_t)slot0 * kMaxGroup + i, (long long)Hk * kMaxGroup,
+                      R.n_split, P.o_d + ((size_t)r * P.H + (size_t)g * G + i) * D,
+                      P.lse_d + (size_t)r * P.H + (size_t)g * G + i, lane);
+  }
+  return true;
+}
+
+// ============================================================= prefill unit
+struct PrefillRange {
+  int req, head, qtile, split;
+  int t0, n;  // first KV tile and number of KV tiles
+};
+
+POD_DEV PrefillRange prefill_range(const Plan& P, int u) {
+  const PrefillUnit U = P.punits[u];
+  const PrefillReq R = P.preq[U.req];
+  const int kv_hi = R.prior + min(R.chunk, (U.qtile + 1) * kQTile);
+  const int n_all = (kv_hi + kKVTile - 1) / kKVTile;
+  PrefillRange pr;
+  pr.req = U.req;
+  pr.head = U.head;
+  pr.qtile = U.qtile;
+  pr.split = U.split;
+  pr.t0 = (int)((long long)U.split * n_all / R.n_split);
+  pr.n = (int)((long long)(U.split + 1) * n_all / R.n_split) - pr.t0;
+  return pr;
+}
+
+// Per-CTA iteration counters that carry mbarrier phases across units.
+struct PipeState {
+  uint32_t kv;  // KV tiles processed
+  uint32_t q;   // Q tiles loaded
+  uint32_t s;   // S tiles (= kv)
+  uint32_t pv;  // PV completions observed by softmax threads
+};
+
+// ---- TMA producer (one thread)
+template <int D>
+POD_DEV bool prefill_producer(const Plan& P, const TmaDescs& T, const PrefillRange& pr,
+                              uint8_t* sm, PipeState& ps, volatile int* abort_flag) {
+  using L = FusedLayout<D>;
+  const uint32_t base = smem_u32(sm);
+  const uint32_t bars = base + L::BAR_OFF;
+  const PrefillReq R = P.preq[pr.req];
+  const int g = pr.head / P.G;
+  constexpr int NB = D / 64;  // 64-column swizzle blocks
+  // Q tile
+  mbar_expect_tx(bars + L::B_Q * 8, L::QB);
+  for (int b = 0; b < NB; ++b)
+    tma_load_3d(base + L::Q_OFF + b * (kQTile * 128), &T.q, bars + L::B_Q * 8, 64 * b, pr.head,
+                R.q_row0 + pr.qtile * kQTile);
+  ps.q++;
+  const CUtensorMap* km = P.paged ? &T.k[0] : &T.k[pr.req];
+  const CUtensorMap* vm = P.paged ? &T.v[0] : &T.v[pr.req];
+  const int last_page = (R.kv_len - 1) >> 4;
+  for (int j = 0; j < pr.n; ++j) {
+    const uint32_t it = ps.kv + j;
+    const uint32_t st = it % kPrefillStages;
+    const uint32_t ph = (it / kPrefillStages) & 1;
+    if (it >= kPrefillStages) {
+      if (!wait_bar(bars + (L::B_KVE + st) * 8, ph ^ 1, P, abort_flag)) {
+        ps.kv += j;
+        return false;
+      }
+    }
+    const int key0 = (pr.t0 + j) * kKVTile;
+    const uint32_t kdst = base + L::K_OFF + st * L::KT;
+    const uint32_t vdst = base + L::V_OFF + st * L::KT;
+    const uint32_t kf = bars + (L::B_KF + st) * 8, vf = bars + (L::B_VF + st) * 8;
+    mbar_expect_tx(kf, L::KT);
+    if (!P.paged) {
+      for (int b = 0; b < NB; ++b) tma_load_3d(kdst + b * (kKVTile * 128), km, kf, 64 * b, g, key0);
+    } else {
+      for (int pg = 0; pg < kKVTile / 16; ++pg) {
+        const int lp = min((key0 >> 4) + pg, last_page);
+        const int phys = __ldg(P.bt_p + (size_t)R.bt_row * P.bt_stride_p + lp);
+        for (int b = 0; b < NB; ++b)
+          tma_load_3d(kdst + b * (kKVTile * 128) + pg * 16 * 128, km, kf, 64 * b, g, phys * 16);
+      }
+    }
+    mbar_expect_tx(vf, L::KT);
+    if (!P.paged) {
+      for (int b = 0; b < NB; ++b) tma_load_3d(vdst + b * (kKVTile * 128), vm, vf, 64 * b, g, key0);
+    } else {
+      for (int pg = 0; pg < kKVTile / 16; ++pg) {
+        const int lp = min((key0 >> 4) + pg, last_page);
+        const int phys = __ldg(P.bt_p + (size_t)R.bt_row * P.bt_stride_p + lp);
+        for (int b = 0; b < NB; ++b)
+          tma_load_3d(vdst + b * (kKVTile * 128) + pg * 16 * 128, vm, vf, 64 * b, g, phys * 16);
+      }
+    }
+  }
+  ps.kv += pr.n;
+  return true;
+}
+
+template <int D>
+POD_DEV void prefill_producer_drain(const Plan& P, uint8_t* sm, const PipeState& ps) {
+  using L = FusedLayout<D>;
+  const uint32_t bars = smem_u32(sm) + L::BAR_OFF;
+  if (ps.q > 0) drain_bar(bars + L::B_Q * 8, (ps.q - 1) & 1, P.wait_budget);
+  for (uint32_t k = 0; k < kPrefillStages && k < ps.kv; ++k) {
+    const uint32_t it = ps.kv - 1 - k;
+    const uint32_t st = it % kPrefillStages, ph = (it / kPrefillStages) & 1;
+    drain_bar(bars + (L::B_KF + st) * 8, ph, P.wait_budget);
+    drain_bar(bars + (L::B_VF + st) * 8, ph, P.wait_budget);
+  }
+}
+
+// ---- MMA issuer (one thread)
+template <int D>
+POD_DEV bool prefill_mma(const Plan& P, const PrefillRange& pr, uint8_t* sm, uint32_t tmem,
+                         PipeState& ps, uint32_t& last_commit_bar, uint32_t& last_commit_par,
+                         volatile int* abort_flag) {
+  using L = FusedLayout<D>;
+  constexpr int KS = D / 16;
+  constexpr uint32_t IDESC_QK = umma_idesc_bf16(kQTile, kKVTile, 0, 0);
+  constexpr uint32_t IDESC_PV = umma_idesc_bf16(kQTile, D, 0, 1);
+  const uint32_t base = smem_u32(sm);
+  const uint32_t bars = base + L::BAR_OFF;
+  if (!wait_bar(bars + L::B_Q * 8, ps.q & 1, P, abort_flag)) return false;
+  ps.q++;
+  tc_fence_after();
+
+  auto issue_pv = [&](int jj) -> bool {
+    const uint32_t it = ps.kv + jj;
+    const uint32_t st = it % kPrefillStages, ph = (it / kPrefillStages) & 1;
+    if (!wait_bar(bars + L::B_PF * 8, it & 1, P, abort_flag)) return false;
+    if (!wait_bar(bars + (L::B_VF + st) * 8, ph, P, abort_flag)) return false;
+    tc_fence_after();
+    const uint32_t pbase = (D >= 128) ? (base + L::K_OFF + st * L::KT) : (base + L::P_OFF);
+    const uint32_t vbase = base + L::V_OFF + st * L::KT;
+#pragma unroll
+    for (int kk = 0; kk < kKVTile / 16; ++kk) {
+      const uint64_t ad = sw128_desc(pbase + kk * 32, 16, 1024);
+      const uint64_t bd = sw128_desc(vbase + kk * 16 * 128, kKVTile * 128, 1024);
+      umma_ss(tmem + 0, ad, bd, IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
+    }
+    umma_commit(bars + L::B_PV * 8);
+    umma_commit(bars + (L::B_KVE + st) * 8);
+    last_commit_bar = bars + L::B_PV * 8;
+    last_commit_par = it & 1;  // pv_done completes once per tile
+    return true;
+  };
+
+  for (int j = 0; j < pr.n; ++j) {
+    const uint32_t it = ps.kv + j;
+    const uint32_t st = it % kPrefillStages, ph = (it / kPrefillStages) & 1;
+    const uint32_t b = it & 1;
+    if (!wait_bar(bars + (L::B_KF + st) * 8, ph, P, abort_flag)) return false;
+    if (it >= 2 && !wait_bar(bars + (L::B_SE + b) * 8, ((it >> 1) - 1) & 1, P, abort_flag))
+      return false;
+    tc_fence_after();
+    const uint32_t kbase = base + L::K_OFF + st * L::KT;
+#pragma unroll
+    for (int kk = 0; kk < KS; ++kk) {
+      const uint64_t ad = sw128_desc(base + L::Q_OFF + (kk >> 2) * (kQTile * 128) + (kk & 3) * 32,
+                                     16, 1024);
+      const uint64_t bd = sw128_desc(kbase + (kk >> 2) * (kKVTile * 128) + (kk & 3) * 32, 16, 1024);
+      umma_ss(tmem + 128 + 64 * b, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
+    }
+    umma_commit(bars + (L::B_SF + b) * 8);
+    last_commit_bar = bars + (L::B_SF + b) * 8;
+    last_commit_par = (it >> 1) & 1;
+    if (j > 0 && !issue_pv(j - 1)) return false;
+  }
+  if (!issue_pv(pr.n - 1)) return false;
+  ps.kv += pr.n;
+  return true;
+}
+
+// ---- softmax + epilogue (128 threads, thread = query row = TMEM lane)
+template <int D>
+POD_DEV bool prefill_softmax(const Plan& P, const PrefillRange& pr, uint8_t* sm, uint32_t tmem,
+                             PipeState& ps, int tid, volatile int* abort_flag, int* s_flag) {
+  using L = FusedLayout<D>;
+  const uint32_t base = smem_u32(sm);
+  const uint32_t bars = base + L::BAR_OFF;
+  const PrefillReq R = P.preq[pr.req];
+  const int warp = tid >> 5;
+  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+  const int row = tid;
+  const int q_local = pr.qtile * kQTile + row;  // token index within the chunk
+  const int lim = R.prior + q_local;            // last visible key (inclusive)
+  const int mask_from = R.prior + pr.qtile * kQTile;  // tiles ending above this need masking
+  const float sc = P.scale_log2;
+  float m_run = -INFINITY, l_run = 0.f;
+  bool failed = false;  // warp-uniform; after a failure only barrier points are kept
+
+  for (int j = 0; j < pr.n; ++j) {
+    const uint32_t it = ps.kv + j;
+    const uint32_t st = it % kPrefillStages;
+    const uint32_t b = it & 1;
+    if (!wait_bar_warp(bars + (L::B_SF + b) * 8, (it >> 1) & 1, P, abort_flag)) {
+      failed = true;
+      break;
+    }
+    tc_fence_after();
+    uint32_t sr[2][32];
+    tmem_ld32(tmem + lane_base + 128 + 64 * b, sr[0]);
+    tmem_ld32(tmem + lane_base + 128 + 64 * b + 32, sr[1]);
+    tc_fence_before();
+    mbar_arrive(bars + (L::B_SE + b) * 8);
+
+    const int key0 = (pr.t0 + j) * kKVTile;
+    float s[64];
+#pragma unroll
+    for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(sr[c >> 5][c & 31]);
+    if (key0 + kKVTile - 1 > mask_from) {
+#pragma unroll
+      for (int c = 0; c < 64; ++c)
+        if (key0 + c > lim) s[c] = -INFINITY;
+    }
+    float mx = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < 64; ++c) mx = fmaxf(mx, s[c]);
+    mx *= sc;
+    // Lazy rescale: keep the reference max unless the tile max exceeds it by
+    // more than 8 (log2 units), which bounds P by 2^8.
+    float alpha = 1.f;
+    bool rescale = false;
+    if (mx > m_run + 8.f) {
+      alpha = ex2(m_run - mx);  // 0 when m_run = -inf
+      rescale = (j > 0) && (m_run != -INFINITY);
+      m_run = mx;
+    }
+    const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+    uint32_t pk[32];
+    float lt = 0.f;
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+      const float p0 = ex2(fmaf(s[2 * c], sc, -m_use));
+      const float p1 = ex2(fmaf(s[2 * c + 1], sc, -m_use));
+      pk[c] = pack_bf16(p0, p1);
+      lt += p0 + p1;  // unrounded weights (see the decode path)
+    }
+    l_run = l_run * alpha + lt;
+    // PV of the previous tile must be done before O is touched (and before
+    // the separate P buffer is overwritten when d < 128).
+    if (j > 0) {
+      if (!wait_bar_warp(bars + L::B_PV * 8, ps.pv & 1, P, abort_flag)) {
+        failed = true;
+        break;
+      }
+      ps.pv++;
+      tc_fence_after();
+    }
+    // tcgen05.ld/st are warp-collective (.sync.aligned): the whole warp takes
+    // this branch if any of its rows must rescale; the others multiply by 1.
+    if (__any_sync(0xffffffffu, rescale)) {
+      const float f = rescale ? alpha : 1.f;
+#pragma unroll
+      for (int cb = 0; cb < D / 32; ++cb) {
+        uint32_t ov[32];
+        tmem_ld32(tmem + lane_base + cb * 32, ov);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * f);
+        tmem_st32(tmem + lane_base + cb * 32, ov);
+      }
+    }
+    // P (bf16, 128 rows x 64 keys, K-major, 128-byte swizzle) into smem.
+    uint8_t* prow = sm + ((D >= 128) ? (L::K_OFF + st * L::KT) : L::P_OFF) + row * 128;
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch) {
+      uint4 v = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+      *reinterpret_cast<uint4*>(prow + ((ch ^ (row & 7)) << 4)) = v;
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    mbar_arrive(bars + L::B_PF * 8);
+  }
+  // final PV
+  if (!failed) {
+    if (wait_bar_warp(bars + L::B_PV * 8, ps.pv & 1, P, abort_flag)) {
+      ps.pv++;
+      tc_fence_after();
+    } else {
+      failed = true;
+    }
+  }
+  ps.kv += pr.n;
+
+  const PrefillReq& RR = R;
+  const bool valid = (q_local < RR.chunk) && !failed;
+  const size_t out_row = (size_t)(RR.q_row0 + q_local);
+  const float lse2 = (l_run > 0.f) ? (m_run + log2f(l_run)) : -INFINITY;
+  if (RR.n_split <= 1) {
+    if (failed) return false;
+    const float inv = 1.f / l_run;
+#pragma unroll
+    for (int cb = 0; cb < D / 32; ++cb) {
+      uint32_t ov[32];
+      tmem_ld32(tmem + lane_base + cb * 32, ov);
+      if (valid) {
+        uint16_t* dst = P.o_p + (out_row * P.H + pr.head) * D + cb * 32;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint4 v;
+          v.x = pack_bf16(__uint_as_float(ov[8 * q + 0]) * inv, __uint_as_float(ov[8 * q + 1]) * inv);
+          v.y = pack_bf16(__uint_as_float(ov[8 * q + 2]) * inv, __uint_as_float(ov[8 * q + 3]) * inv);
+          v.z = pack_bf16(__uint_as_float(ov[8 * q + 4]) * inv, __uint_as_float(ov[8 * q + 5]) * inv);
+          v.w = pack_bf16(__uint_as_float(ov[8 * q + 6]) * inv, __uint_as_float(ov[8 * q + 7]) * inv);
+          *reinterpret_cast<uint4*>(dst + 8 * q) = v;
+        }
+      }
+    }
+    if (valid) P.lse_p[out_row * P.H + pr.head] = lse2 * kLn2;
+    return true;
+  }
+  // split partial: normalised O (fp32) and LSE of this KV range
+  const int gidx = pr.qtile * P.H + pr.head;
+  const int slot = RR.slot0 + gidx * RR.n_split + pr.split;
+  const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
+  float* po = P.ppart_o + ((size_t)slot * kQTile + row) * D;
+#pragma unroll
+  for (int cb = 0; cb < D / 32 && !failed; ++cb) {
+    uint32_t ov[32];
+    tmem_ld32(tmem + lane_base + cb * 32, ov);
+    if (valid) {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        float4 v = make_float4(__uint_as_float(ov[4 * q]) * inv, __uint_as_float(ov[4 * q + 1]) * inv,
+                               __uint_as_float(ov[4 * q + 2]) * inv,
+                               __uint_as_float(ov[4 * q + 3]) * inv);
+        *reinterpret_cast<float4*>(po + cb * 32 + 4 * q) = v;
+      }
+    }
+  }
+  if (valid) P.ppart_lse[(size_t)slot * kQTile + row] = lse2 * kLn2;
+  __threadfence();
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+  if (tid == 0) {
+    // after a failure nobody merges (the group can never be complete)
+    const int old = *abort_flag ? -1 : atomicAdd(P.pgroup_ctr + RR.group0 + gidx, 1);
+    *s_flag = (old == RR.n_split - 1);
+  }
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+  if (*s_flag && !failed) {
+    __threadfence();
+    const int rows = min(kQTile, RR.chunk - pr.qtile * kQTile);
+    const int slot0 = RR.slot0 + gidx * RR.n_split;
+    for (int rr = warp; rr < rows; rr += 4) {
+      const size_t orow = (size_t)(RR.q_row0 + pr.qtile * kQTile + rr);
+      merge_row_warp<D>(P.ppart_o + ((size_t)slot0 * kQTile + rr) * D, (long long)kQTile * D,
+                        P.ppart_lse + (size_t)slot0 * kQTile + rr, kQTile, RR.n_split,
+                        P.o_p + (orow * P.H + pr.head) * D, P.lse_p + orow * P.H + pr.head,
+                        tid & 31);
+    }
+  }
+  return !failed;
+}
+
+// ============================================================= fused kernel
+// Roles: PREFILL = 1, DECODE = 2. allow_prefill / allow_decode restrict the
+// queues (prefill-only launch = allow_decode 0).
+template <int D>
+__global__ void __launch_bounds__(kFusedThreads, kFusedSlotsPerSm)
+    pod_fused_kernel(const __grid_constant__ Plan P, const __grid_constant__ TmaDescs T,
+                     int allow_prefill, int allow_decode) {
+  using L = FusedLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~(uintptr_t)1023);
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const uint32_t bars = smem_u32(sm) + L::BAR_OFF;
+  int* misc = reinterpret_cast<int*>(sm + L::MISC_OFF);
+  // misc[0] tmem addr, [1] role, [2] unit, [3] abort flag, [4] merge flag,
+  // [5] prefill queue empty, [6] decode queue empty
+  volatile int* abort_flag = misc + 3;
+
+  if (tid == 0) {
+    for (int i = 0; i < L::N_BARS; ++i) {
+      uint32_t cnt = 1;
+      if (i == L::B_SE || i == L::B_SE + 1 || i == L::B_PF) cnt = 128;
+      mbar_init(bars + i * 8, cnt);
+    }
+    fence_mbar_init();
+    misc[3] = 0;
+    misc[5] = allow_prefill ? 0 : 1;
+    misc[6] = allow_decode ? 0 : 1;
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(misc), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = static_cast<uint32_t>(misc[0]);
+
+  // Test hook: one thread waits on a flag nothing sets, with a short budget,
+  // then records the timeout and carries on.
+  if ((P.flags & 0x2) && blockIdx.x == 0 && tid == 0) {
+    const long long t0 = clock64();
+    while (*reinterpret_cast<volatile const int*>(P.never_set) == 0) {
+      if (clock64() - t0 > 2000000LL) {
+        set_status(P, kStatusTimeout);
+        break;
+      }
+    }
+  }
+
+  const uint32_t my_sm = smid() & (kMaxSmid - 1);
+  PipeState ps = {0u, 0u, 0u, 0u};
+  uint32_t dec_ring = 0;
+  uint32_t last_commit_bar = 0, last_commit_par = 0;
+  bool issued_mma = false;
+
+  while (true) {
+    if (tid == 0) {
+      int role = 0, unit = -1;
+      if (!*abort_flag) {
+        const int t = atomicAdd(P.sm_ticket + my_sm, 1);
+        const long long num = P.rho_num, den = P.rho_den > 0 ? P.rho_den : 1;
+        bool want_p = ((long long)(t + 1) * num) / den > ((long long)t * num) / den;
+        for (int attempt = 0; attempt < 2 && role == 0; ++attempt, want_p = !want_p) {
+          if (want_p && !misc[5]) {
+            const int u = atomicAdd(P.ctl + 0, 1);
+            if (u < P.n_prefill_units) {
+              role = 1;
+              unit = u;
+            } else {
+              misc[5] = 1;
+            }
+          } else if (!want_p && !misc[6]) {
+            const int u = atomicAdd(P.ctl + 1, kFusedWarps);
+            if (u < P.n_decode_units) {
+              role = 2;
+              unit = u;
+            } else {
+              misc[6] = 1;
+            }
+          }
+        }
+        if (role && (P.flags & 0x1)) atomicAdd(P.stats + my_sm * 2 + (role - 1), 1);
+      }
+      misc[1] = role;
+      misc[2] = unit;
+    }
+    __syncthreads();
+    const int role = misc[1];
+    const int unit = misc[2];
+    if (role == 0) break;
+    if (role == 1) {
+      const PrefillRange pr = prefill_range(P, unit);
+      if (warp < 4) {
+        prefill_softmax<D>(P, pr, sm, tmem, ps, tid, abort_flag, misc + 4);
+      } else if (warp == 4) {
+        if (lane == 0) {
+          issued_mma = true;
+          prefill_mma<D>(P, pr, sm, tmem, ps, last_commit_bar, last_commit_par, abort_flag);
+        }
+        __syncwarp();
+      } else {
+        if (lane == 0) prefill_producer<D>(P, T, pr, sm, ps, abort_flag);
+        __syncwarp();
+      }
+    } else {
+      const int u = unit + warp;
+      if (u < P.n_decode_units) {
+        decode_unit_warp<D, kFusedDecStages>(P, u, sm + warp * L::DEC_WARP,
+                                             bars + (L::B_DEC + warp * kFusedDecStages) * 8,
+                                             dec_ring, lane, true, abort_flag);
+      }
+    }
+    __syncthreads();
+    if (*abort_flag) break;
+  }
+  // Teardown. After an abort, wait (bounded) for this CTA's own async work.
+  if (*abort_flag) {
+    if (warp == 5 && lane == 0) prefill_producer_drain<D>(P, sm, ps);
+    if (warp == 4 && lane == 0 && issued_mma && last_commit_bar)
+      drain_bar(last_commit_bar, last_commit_par, P.wait_budget);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ============================================================= decode-only kernels
+template <int D>
+__global__ void __launch_bounds__(kDecodeWarps * 32)
+    pod_decode_kernel(const __grid_constant__ Plan P) {
+  using L = DecodeLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 15) &
+                                           ~(uintptr_t)15);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int u = blockIdx.x * kDecodeWarps + warp;
+  if (u >= P.n_decode_units) return;
+  const uint32_t bar0 = smem_u32(sm + L::BAR_OFF) + warp * kDecodeStages * 8;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::BAR_OFF +
+                                                              kDecodeWarps * kDecodeStages * 8) +
+                             warp;
+  if (lane == 0) {
+    for (int i = 0; i < kDecodeStages; ++i) mbar_init(bar0 + i * 8, 1);
+    fence_mbar_init();
+    *abort_flag = 0;
+  }
+  __syncwarp();
+  uint32_t ring = 0;
+  decode_unit_warp<D, kDecodeStages>(P, u, sm + warp * L::WARP, bar0, ring, lane, false, abort_flag);
+}
+
+// One warp per (decode request, query head) whose KV range was split.
+template <int D>
+__global__ void __launch_bounds__(128) pod_merge_kernel(const __grid_constant__ Plan P) {
+  const int gw = blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (gw >= P.n_decode_reqs * P.H) return;
+  const int r = gw / P.H, h = gw - (gw / P.H) * P.H;
+  const DecodeReq R = P.dreq[r];
+  if (R.n_split <= 1) return;
+  const int g = h / P.G, i = h - (h / P.G) * P.G;
+  const int slot0 = R.slot0 + g;
+  merge_row_warp<D>(P.dpart_o + ((size_t)slot0 * kMaxGroup + i) * D,
+                    (long long)P.Hk * kMaxGroup * D, P.dpart_lse + (size_t)slot0 * kMaxGroup + i,
+                    (long long)P.Hk * kMaxGroup, R.n_split, P.o_d + ((size_t)r * P.H + h) * D,
+                    P.lse_d + (size_t)r * P.H + h, lane);
+}
+
+// ============================================================= host-side launchers
+template <int D>
+static cudaError_t set_attrs() {
+  cudaError_t e = cudaFuncSetAttribute(pod_fused_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       FusedLayout<D>::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(pod_decode_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              DecodeLayout<D>::SMEM_BYTES);
+}
+
+cudaError_t kernels_init(int D) { return D == 128 ? set_attrs<128>() : set_attrs<64>(); }
+
+int fused_smem_bytes(int D) {
+  return D == 128 ? FusedLayout<128>::SMEM_BYTES : FusedLayout<64>::SMEM_BYTES;
+}
+int decode_smem_bytes(int D) {
+  return D == 128 ? DecodeLayout<128>::SMEM_BYTES : DecodeLayout<64>::SMEM_BYTES;
+}
+
+cudaError_t launch_fused(const Plan& P, const TmaDescs& T, int grid, int allow_prefill,
+                         int allow_decode, cudaStream_t s) {
+  if (P.D == 128)
+    pod_fused_kernel<128><<<grid, kFusedThreads, FusedLayout<128>::SMEM_BYTES, s>>>(
+        P, T, allow_prefill, allow_decode);
+  else
+    pod_fused_kernel<64><<<grid, kFusedThreads, FusedLayout<64>::SMEM_BYTES, s>>>(
+        P, T, allow_prefill, allow_decode);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode(const Plan& P, cudaStream_t s) {
+  const int grid = (P.n_decode_units + kDecodeWarps - 1) / kDecodeWarps;
+  if (grid == 0) return cudaSuccess;
+  if (P.D == 128)
+    pod_decode_kernel<128><<<grid, kDecodeWarps * 32, DecodeLayout<128>::SMEM_BYTES, s>>>(P);
+  else
+    pod_decode_kernel<64><<<grid, kDecodeWarps * 32, DecodeLayout<64>::SMEM_BYTES, s>>>(P);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_merge(const Plan& P, cudaStream_t s) {
+  const int rows = P.n_decode_reqs * P.H;
+  const int grid = (rows + 3) / 4;
+  if (grid == 0) return cudaSuccess;
+  if (P.D == 128)
+    pod_merge_kernel<128><<<grid, 128, 0, s>>>(P);
+  else
+    pod_merge_kernel<64><<<grid, 128, 0, s>>>(P);
+  return cudaGetLastError();
+}
+
+}  // namespace pod

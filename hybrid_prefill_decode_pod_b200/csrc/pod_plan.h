@@ -1,0 +1,92 @@
+// pod_plan.h -- work-unit plan shared by the host planner and the kernels.
+//
+// The planner splits a hybrid batch into independent work units (POD-Attention
+// §4 "POD-Attention": prefill and decode CTAs are remapped onto the device
+// functions of the two phases; §4.2.3 caps chunked-prefill splits at two full
+// waves; the persistent-thread form of §4.4 pulls units from queues):
+//   prefill unit = (request, query head, 128-row query tile, KV split)
+//   decode unit  = (request, KV head, KV split of `dec_split_len` keys)
+// Units whose KV range is split write fp32 partial results and are merged by
+// log-sum-exp in split order, so results never depend on which CTA ran what.
+#pragma once
+#include <cuda.h>
+#include <stdint.h>
+
+namespace pod {
+
+constexpr int kMaxPrefillReqs = 16;
+constexpr int kQTile = 128;           // prefill query rows per unit (= UMMA M)
+constexpr int kKVTile = 64;           // prefill keys per KV tile (= UMMA N of S)
+constexpr int kPrefillStages = 2;     // K/V smem ring depth in the prefill role
+constexpr int kDecTile = 16;          // decode keys per staged tile (= mma M)
+constexpr int kFusedWarps = 6;        // 4 softmax + 1 MMA issuer + 1 TMA producer
+constexpr int kFusedThreads = kFusedWarps * 32;
+constexpr int kFusedSlotsPerSm = 2;   // persistent CTAs per SM
+constexpr int kFusedDecStages = 2;    // per-warp decode ring depth in the fused kernel
+constexpr int kDecodeWarps = 4;       // warps (virtual decode units) per decode-only CTA
+constexpr int kDecodeStages = 3;      // per-warp ring depth in the decode-only kernel
+constexpr int kMaxGroup = 8;          // query heads per KV head (mma N = 8)
+constexpr int kTmemCols = 256;        // TMEM columns per CTA: O [0,128), S0, S1 [128,256)
+constexpr int kMaxSmid = 256;         // per-SM ticket slots (indexed by %smid)
+constexpr long long kDefaultWaitBudget = 2000000000LL;  // cycles (~1 s at 2 GHz)
+
+struct PrefillReq {
+  int prior, chunk, q_row0, n_qtiles;
+  int kv_len, bt_row, n_split, group0;  // group0: first merge group of this request
+  int slot0, n_kvtiles_max, pad0, pad1; // slot0: first partial slot (split requests)
+};
+
+struct PrefillUnit {
+  int req, head, qtile, split;
+};
+
+struct DecodeReq {
+  const uint16_t* k;  // contiguous caches (null when paged)
+  const uint16_t* v;
+  int len, n_split, unit0, slot0;   // slot0: first partial slot (split requests)
+  int group0, bt_row, pad0, pad1;
+};
+
+// Kernel parameters (by value). Pointers refer to the device workspace or to
+// the caller's tensors.
+struct Plan {
+  int H, Hk, G, D;
+  float scale_log2;              // log2(e) / sqrt(d)
+  int n_prefill_units, n_decode_units, n_prefill_reqs, n_decode_reqs;
+  int dec_split_len;
+  int rho_num, rho_den;          // prefill share of claims (per-SM Bresenham)
+  int paged;
+  int bt_stride_p, bt_stride_d;
+  int flags;
+  int pool_blocks;               // paged: blocks in the pool (bounds every block id)
+  long long wait_budget;         // cycles a bounded wait may spin
+  const PrefillReq* preq;
+  const PrefillUnit* punits;
+  const DecodeReq* dreq;
+  const int* dunit_req;          // request of each decode unit
+  const uint16_t* q_p; uint16_t* o_p; float* lse_p;
+  const uint16_t* q_d; uint16_t* o_d; float* lse_d;
+  const int* bt_p; const int* bt_d;
+  const uint16_t* k_pool; const uint16_t* v_pool;
+  float* ppart_o; float* ppart_lse;   // prefill partials [slot][128][d], [slot][128]
+  float* dpart_o; float* dpart_lse;   // decode partials  [slot][8][d],   [slot][8]
+  int* ctl;                           // [0] prefill queue head, [1] decode queue head
+  int* sm_ticket;                     // [kMaxSmid]
+  int* pgroup_ctr;                    // arrivals per prefill merge group
+  int* dgroup_ctr;                    // arrivals per decode merge group
+  int* stats;                         // [kMaxSmid][2] claims per role (POD_FLAG_STATS)
+  int* status;                        // sticky status word (not reset per call)
+  const int* never_set;               // test-only flag that nothing writes
+};
+
+// Tensor maps for TMA, passed as a __grid_constant__ kernel parameter.
+// Contiguous layout: k[p] / v[p] map request p's [len, Hk, d] cache with a
+// 64-key box. Paged layout: k[0] / v[0] map the pool as [blocks*16, Hk, d]
+// with a 16-key (one page) box.
+struct TmaDescs {
+  CUtensorMap q;
+  CUtensorMap k[kMaxPrefillReqs];
+  CUtensorMap v[kMaxPrefillReqs];
+};
+
+}  // namespace pod

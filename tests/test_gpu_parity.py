@@ -1,0 +1,185 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Tolerances (bf16 outputs vs fp64): O max-abs <= 1e-2 and relative L2 <= 5e-3;
+LSE max-abs <= 1e-3. Scaled-down shapes are compared element by element;
+the full-size configurations (the benchmark's launch configuration) on
+sampled rows the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from hybrid_prefill_decode_pod_b200 import workloads as W
+from hybrid_prefill_decode_pod_b200 import pod_attn as pa
+
+from gpu_util import bitwise_equal, compare, run, sample_indices
+
+pytestmark = pytest.mark.gpu
+
+
+def test_tiny_config_all_modes_match_oracle():
+    b = W.make_batch(W.CONFIGS["tiny"])
+    ref = oracle.hybrid(b)
+    outs = {}
+    for mode in ("fused", "serial", "two_stream"):
+        outs[mode], _ = run(b, mode)
+        compare(ref, outs[mode])
+    assert bitwise_equal(outs["fused"], outs["serial"])
+    assert bitwise_equal(outs["fused"], outs["two_stream"])
+
+
+SHAPES = [
+    # (H, Hk, d, prefill[(prior, chunk)], decode ctx) -- several tiles, ragged tails
+    (8, 2, 128, [(300, 200)], [1, 17, 64, 65, 1000, 3000]),
+    (16, 2, 128, [(0, 130), (77, 257)], [5, 4096, 513]),          # G = 8, prior 0, 2 chunks
+    (4, 4, 128, [(1000, 64)], [2048, 31]),                        # G = 1
+    (8, 4, 64, [(129, 129)], [128, 129, 700]),                    # d = 64, G = 2
+    (32, 8, 128, [(4096, 512)], [4096] * 4),                      # llama-3-8B rows
+]
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+@pytest.mark.parametrize("mode", ["fused", "serial"])
+def test_scaled_shapes_match_oracle(shape, mode):
+    H, Hk, d, pre, ctx = shape
+    b = W.make_custom(H, Hk, d, pre, ctx, seed=5)
+    ref = oracle.hybrid(b)
+    out, plan = run(b, mode)
+    compare(ref, out)
+
+
+def test_paged_matches_contiguous_bitwise_and_oracle():
+    b = W.make_custom(8, 2, 128, [(333, 190), (0, 40)], [1, 16, 17, 999, 2500], seed=9,
+                      paged=True)
+    ref = oracle.hybrid(b)
+    paged, _ = run(b, "fused", paged=True)
+    contig, _ = run(b, "fused", paged=False)
+    compare(ref, paged)
+    assert bitwise_equal(paged, contig)
+
+
+def test_run_to_run_bitwise_and_modes_bitwise():
+    b = W.make_custom(8, 2, 128, [(2000, 300)], [100, 5000, 7000, 64], seed=13)
+    a1, _ = run(b, "fused")
+    a2, _ = run(b, "fused")
+    s1, _ = run(b, "serial")
+    t1, _ = run(b, "two_stream")
+    assert bitwise_equal(a1, a2)
+    assert bitwise_equal(a1, s1)
+    assert bitwise_equal(a1, t1)
+
+
+def test_prefill_only_and_decode_only_match_hybrid():
+    b = W.make_custom(8, 2, 128, [(700, 300)], [3000, 20], seed=17)
+    h, _ = run(b, "fused")
+    p, _ = run(b, "prefill_only")
+    d, _ = run(b, "decode_only")
+    assert torch.equal(h["prefill_o"].view(torch.int16), p["prefill_o"].view(torch.int16))
+    assert torch.equal(h["decode_o"].view(torch.int16), d["decode_o"].view(torch.int16))
+    assert torch.equal(h["decode_lse"], d["decode_lse"])
+
+
+def test_invariants_on_gpu():
+    """Constant V returns V; K == 0 gives ln(#keys); one key returns its V."""
+    b = W.make_custom(8, 2, 128, [(0, 150)], [1, 200, 3000], seed=21)
+    for v in b.v_prefill + b.v_decode:
+        v[:, 0] = 0.5
+        v[:, 1] = -2.0
+    for k in b.k_prefill + b.k_decode:
+        k.zero_()
+    out, _ = run(b, "fused")
+    c = torch.tensor([0.5] * 4 + [-2.0] * 4)
+    # P is rounded to bf16 for the tensor cores, the normaliser is not: within
+    # one bf16 ulp of |c| (the rows-sum-to-one invariant on the GPU).
+    tol = c.abs()[None, :, None] * 2.0 ** -7
+    assert ((out["decode_o"].float() - c[None, :, None]).abs() <= tol).all()
+    assert ((out["prefill_o"].float() - c[None, :, None]).abs() <= tol).all()
+    for r, L in enumerate(b.ctx):
+        assert np.abs(out["decode_lse"][r].numpy() - np.log(L)).max() < 1e-5
+    t = np.arange(150)
+    assert np.abs(out["prefill_lse"].numpy() - np.log(t + 1)[:, None]).max() < 1e-5
+    # single key: decode L = 1 returns V0 bitwise
+    b2 = W.make_custom(8, 2, 128, [], [1, 1], seed=23)
+    out2, _ = run(b2, "fused")
+    for r in range(2):
+        for h in range(8):
+            assert torch.equal(out2["decode_o"][r, h], b2.v_decode[r][0, h // 4])
+
+
+def test_causal_mask_on_gpu():
+    """Changing K/V at position P leaves rows with prior + t < P bitwise unchanged."""
+    prior, c = 200, 300
+    b = W.make_custom(8, 2, 128, [(prior, c)], [], seed=29)
+    a, _ = run(b, "fused")
+    P = prior + 123
+    b.k_prefill[0][P] = 3.0
+    b.v_prefill[0][P] = -3.0
+    a2, _ = run(b, "fused")
+    assert torch.equal(a["prefill_o"][:123].view(torch.int16), a2["prefill_o"][:123].view(torch.int16))
+    assert not torch.equal(a["prefill_o"][123:].view(torch.int16), a2["prefill_o"][123:].view(torch.int16))
+
+
+def test_decode_permutation_permutes_outputs():
+    b = W.make_custom(8, 2, 128, [], [5, 8000, 333, 1], seed=31)
+    a, _ = run(b, "fused")
+    perm = [2, 0, 3, 1]
+    b2 = W.make_custom(8, 2, 128, [], [b.ctx[i] for i in perm], seed=31)
+    b2.q_decode = b.q_decode[perm].clone()
+    b2.k_decode = [b.k_decode[i] for i in perm]
+    b2.v_decode = [b.v_decode[i] for i in perm]
+    a2, _ = run(b2, "fused")
+    assert torch.equal(a2["decode_o"].view(torch.int16), a["decode_o"][perm].view(torch.int16))
+
+
+def test_empty_sides():
+    b = W.make_custom(8, 2, 128, [(10, 0)], [50], seed=37)      # chunk 0 is a no-op
+    ref = oracle.hybrid(b)
+    out, _ = run(b, "fused")
+    compare(ref, out, keys=("decode",))
+    b2 = W.make_custom(8, 2, 128, [(10, 70)], [], seed=37)      # no decodes
+    out2, _ = run(b2, "fused")
+    compare(oracle.hybrid(b2), out2, keys=("prefill",))
+
+
+def test_timeout_path_reports_status_and_keeps_results():
+    b = W.make_custom(8, 2, 128, [(64, 64)], [100], seed=41)
+    pod = pa.context_for(b, flags=pa.FLAG_TEST_FORCE_TIMEOUT)
+    db = pa.DeviceBatch(b)
+    pre, dec = db.args(pod)
+    pod.hybrid(pre, dec, pa.MODE_FUSED)
+    assert pod.status() == pa.POD_ETIMEOUT
+    assert pod.status() == pa.POD_OK       # cleared by the read
+    out = {"prefill_o": db.o_p.cpu(), "prefill_lse": db.lse_p.cpu(),
+           "decode_o": db.o_d.cpu(), "decode_lse": db.lse_d.cpu()}
+    compare(oracle.hybrid(b), out)
+    assert pod.close() == pa.POD_OK
+
+
+def test_stats_show_both_roles_per_sm():
+    b = W.make_batch(W.CONFIGS["llama3_8b"])
+    pod = pa.context_for(b, flags=pa.FLAG_STATS)
+    db = pa.DeviceBatch(b)
+    pre, dec = db.args(pod)
+    pod.hybrid(pre, dec, pa.MODE_FUSED)
+    st = pod.stats()
+    plan = pod.last_plan()
+    assert st["prefill_claims"] == plan["prefill_units"]
+    assert st["sms_with_both"] > plan["num_sms"] // 2
+    pod.close()
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["llama3_8b", "decode_heavy", "long_context", "paged"])
+def test_full_size_configs_sampled(name):
+    """Full-size configuration, FUSED launch as benchmarked; oracle on sampled rows."""
+    b = W.make_batch(W.CONFIGS[name])
+    H = b.cfg.num_qo_heads
+    ps = sample_indices(b.total_prefill_tokens, H, 192, 1)
+    ds = sample_indices(b.num_decodes, H, 192, 2)
+    ref = oracle.hybrid(b, prefill_sample=ps, decode_sample=ds)
+    out, plan = run(b, "fused")
+    compare(ref, out, sample={"prefill": ps, "decode": ds})
+    # properties at any size: finite everywhere, LSE >= max score bound sanity
+    for k in ("prefill_o", "decode_o", "prefill_lse", "decode_lse"):
+        assert torch.isfinite(out[k].float()).all(), k
