@@ -190,8 +190,10 @@ def oracle_sample_time(batch, budget_s: float, seed: int = 0):
     for _ in range(6):
         np_items = max(1, int(len(pk) * H * frac))
         nd_items = max(1, int(len(dk) * H * frac)) if len(dk) else 0
-        ps = rng.integers(0, max(1, len(pk) * H), size=np_items) if len(pk) else None
-        ds = rng.integers(0, len(dk) * H, size=nd_items) if len(dk) else None
+        np_items = min(np_items, len(pk) * H)
+        nd_items = min(nd_items, len(dk) * H)
+        ps = np.sort(rng.choice(len(pk) * H, size=np_items, replace=False)) if len(pk) else None
+        ds = np.sort(rng.choice(len(dk) * H, size=nd_items, replace=False)) if len(dk) else None
         t0 = time.perf_counter()
         oracle.hybrid(batch, prefill_sample=ps, decode_sample=ds)
         dt = time.perf_counter() - t0
@@ -199,7 +201,9 @@ def oracle_sample_time(batch, budget_s: float, seed: int = 0):
         spent += dt
         if dt > budget_s * 0.3 or spent > budget_s:
             break
-        frac *= max(2.0, min(8.0, budget_s * 0.4 / max(dt, 1e-3)))
+        if frac >= 0.25:
+            break
+        frac = min(0.25, frac * max(2.0, min(8.0, budget_s * 0.4 / max(dt, 1e-3))))
     us = dt / max(keys, 1) * total_keys * 1e6
     desc = ("%d prefill + %d decode (row, head) items drawn at random (%.3g%% of the keys), "
             "scaled to one call by key count; fp64, %d OpenMP threads"
@@ -211,7 +215,7 @@ def oracle_sample_time(batch, budget_s: float, seed: int = 0):
 def run_reference(args, rank, world):
     if rank != 0:
         return 0
-    batch = W.make_batch(W.CONFIGS[args.workload])
+    batch = W.make_batch(W.get_config(args.workload))
     vals = []
     for i in range(args.warmup + args.steps):
         budget = 0.5 if i < args.warmup else args.ref_step_seconds
@@ -254,7 +258,7 @@ def run_gpu(args, rank, world, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     peaks, peak_kind = load_peaks()
-    cfg = W.CONFIGS[args.workload]
+    cfg = W.get_config(args.workload)
     batch = W.make_batch(cfg)
     paged = cfg.paged
     pod = pa.context_for(batch, device=local, flags=pa.FLAG_STATS if args.stats else 0)
@@ -432,7 +436,7 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.CONFIGS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.CONFIGS) + sorted(W.PROBE_CONFIGS))
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-step-seconds", type=float, default=2.0)
     ap.add_argument("--e2e-steps", type=int, default=10)

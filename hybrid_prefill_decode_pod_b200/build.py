@@ -15,7 +15,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libpod_attn.so")
 SOURCES = [os.path.join(CSRC, "pod_kernels.cu"), os.path.join(CSRC, "pod_attn_api.cpp")]
-HEADERS = [os.path.join(CSRC, f) for f in ("pod_plan.h", "pod_ptx.cuh")] + [
+HEADERS = [os.path.join(CSRC, f) for f in ("pod_plan.h", "pod_ptx.cuh", "pod_exp2.cuh")] + [
     os.path.join(INCLUDE, "pod_attn.h")]
 
 NVCC_FLAGS = [
@@ -42,7 +42,10 @@ def _stale() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False, extra=()) -> str:
-    if not force and not _stale():
+    """Compile the library. POD_ATTN_NVCC_EXTRA (space-separated) adds flags,
+    e.g. -DPOD_SOFT_EXP2_PAIRS=4, for tuning builds."""
+    extra = list(extra) + os.environ.get("POD_ATTN_NVCC_EXTRA", "").split()
+    if not force and not _stale() and not os.environ.get("POD_ATTN_NVCC_EXTRA"):
         return LIB
     tmp = LIB + ".tmp.%d" % os.getpid()
     cmd = [nvcc(), *NVCC_FLAGS, *extra, "-shared", "-o", tmp, *SOURCES, "-lcudart"]

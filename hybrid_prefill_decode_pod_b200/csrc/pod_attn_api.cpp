@@ -29,7 +29,8 @@ int fused_smem_bytes(int D);
 int decode_smem_bytes(int D);
 cudaError_t launch_fused(const Plan& P, const TmaDescs& T, int grid, int allow_prefill,
                          int allow_decode, cudaStream_t s);
-cudaError_t launch_decode(const Plan& P, cudaStream_t s);
+cudaError_t launch_decode(const Plan& P, int max_grid, cudaStream_t s);
+cudaError_t decode_occupancy(int D, int* blocks_per_sm);
 cudaError_t launch_merge(const Plan& P, cudaStream_t s);
 }  // namespace pod
 
@@ -69,6 +70,7 @@ struct PlanLayout {
 struct pod_attn_ctx {
   pod_attn_config cfg{};
   int device = 0, num_sms = 0, slots_per_sm = kFusedSlotsPerSm;
+  int decode_grid = 0;  // persistent decode-only grid (SMs x resident CTAs)
   int H = 0, Hk = 0, G = 0, D = 0;
   int cap_punits = 0, cap_pgroups = 0, cap_pslots = 0;
   int cap_dunits = 0, cap_dgroups = 0, cap_dslots = 0, cap_dreqs = 0;
@@ -485,6 +487,9 @@ int pod_attn_create(pod_attn_ctx** out, const pod_attn_config* cfg) {
     return code;
   };
   if (kernels_init(D) != cudaSuccess) return fail(POD_ECUDA);
+  int dec_blocks = 0;
+  if (decode_occupancy(D, &dec_blocks) != cudaSuccess || dec_blocks < 1) return fail(POD_ECUDA);
+  c->decode_grid = c->num_sms * dec_blocks;
 
   // capacities
   const int slots = c->num_sms * c->slots_per_sm;
@@ -566,7 +571,7 @@ int pod_attn_hybrid(pod_attn_ctx* c, const pod_prefill_args* pa, const pod_decod
   if (mode == POD_MODE_SERIAL) {
     if (has_p && launch_fused(P, T, fused_grid(c, P, false), 1, 0, s) != cudaSuccess)
       return POD_ECUDA;
-    if (has_d && (launch_decode(P, s) != cudaSuccess || launch_merge(P, s) != cudaSuccess))
+    if (has_d && (launch_decode(P, c->decode_grid, s) != cudaSuccess || launch_merge(P, s) != cudaSuccess))
       return POD_ECUDA;
     return POD_OK;
   }
@@ -575,7 +580,7 @@ int pod_attn_hybrid(pod_attn_ctx* c, const pod_prefill_args* pa, const pod_decod
   if (cudaStreamWaitEvent(c->side, c->ev_fork, 0) != cudaSuccess) return POD_ECUDA;
   if (has_p && launch_fused(P, T, fused_grid(c, P, false), 1, 0, s) != cudaSuccess)
     return POD_ECUDA;
-  if (has_d && (launch_decode(P, c->side) != cudaSuccess || launch_merge(P, c->side) != cudaSuccess))
+  if (has_d && (launch_decode(P, c->decode_grid, c->side) != cudaSuccess || launch_merge(P, c->side) != cudaSuccess))
     return POD_ECUDA;
   if (cudaEventRecord(c->ev_join, c->side) != cudaSuccess) return POD_ECUDA;
   if (cudaStreamWaitEvent(s, c->ev_join, 0) != cudaSuccess) return POD_ECUDA;
@@ -610,7 +615,7 @@ int pod_attn_decode_only(pod_attn_ctx* c, const pod_decode_args* da, void* strea
   rc = stage_plan(c, nullptr, da, s, &P, &T);
   if (rc) return rc;
   if (P.n_decode_units == 0) return POD_OK;
-  if (launch_decode(P, s) != cudaSuccess || launch_merge(P, s) != cudaSuccess) return POD_ECUDA;
+  if (launch_decode(P, c->decode_grid, s) != cudaSuccess || launch_merge(P, s) != cudaSuccess) return POD_ECUDA;
   return POD_OK;
 }
 

@@ -23,14 +23,31 @@
 #include <math.h>
 #include <stdint.h>
 
+#include "pod_exp2.cuh"
 #include "pod_plan.h"
 #include "pod_ptx.cuh"
 
 namespace pod {
 
+// Share of the prefill softmax's exponentials evaluated by exp2_poly on the
+// FMA pipe instead of MUFU (pairs out of 8), and the bf16 packing used for P.
+// Measured on B200 (long-context prefill, 64/8 heads, d 128): 0 pairs with
+// cvt packing is fastest (628 us); 2/3/4 pairs gave 687/717/753 us and integer
+// packing 850 us -- this softmax is bound by issue and latency, not by MUFU.
+#ifndef POD_SOFT_EXP2_PAIRS
+#define POD_SOFT_EXP2_PAIRS 0
+#endif
+constexpr int kSoftPairs = POD_SOFT_EXP2_PAIRS;
+#ifndef POD_INT_PACK
+#define POD_PACK(a, b) pack_bf16(a, b)
+#else
+#define POD_PACK(a, b) pack_bf16_int(a, b)
+#endif
+
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kStatusTimeout = -5;
+constexpr int kStatusUnsupported = -2;
 
 POD_DEV void set_status(const Plan& P, int code) { atomicCAS(P.status, 0, code); }
 
@@ -71,12 +88,12 @@ template <int D>
 struct FusedLayout {
   static constexpr int QB = kQTile * D * 2;   // Q tile bytes
   static constexpr int KT = kKVTile * D * 2;  // one K (or V) tile
+  static constexpr int PB = kQTile * kKVTile * 2;  // P tile (bf16)
   static constexpr int Q_OFF = 0;
-  static constexpr int K_OFF = Q_OFF + QB;
-  static constexpr int V_OFF = K_OFF + kPrefillStages * KT;
-  static constexpr int P_OFF = V_OFF + kPrefillStages * KT;  // own P buffer only when d < 128
-  static constexpr int P_BYTES = (D >= 128) ? 0 : kQTile * kKVTile * 2;
-  static constexpr int PREFILL_END = P_OFF + P_BYTES;
+  static constexpr int K_OFF = Q_OFF + QB;                      // K ring
+  static constexpr int V_OFF = K_OFF + kPrefillStages * KT;     // V ring
+  static constexpr int P_OFF = V_OFF + kPrefillStages * KT;     // P (own buffer)
+  static constexpr int PREFILL_END = P_OFF + PB;
   static constexpr int DEC_ROW = D * 2 + 16;  // padded row: conflict-free ldmatrix
   static constexpr int DEC_STAGE = 2 * kDecTile * DEC_ROW;
   static constexpr int DEC_WARP = kFusedDecStages * DEC_STAGE;
@@ -85,10 +102,11 @@ struct FusedLayout {
   static constexpr int BAR_OFF = (DATA_END + 127) & ~127;
   // barrier indices
   static constexpr int B_Q = 0;
-  static constexpr int B_KF = 1;
-  static constexpr int B_VF = B_KF + kPrefillStages;
-  static constexpr int B_KVE = B_VF + kPrefillStages;
-  static constexpr int B_SF = B_KVE + kPrefillStages;
+  static constexpr int B_KF = 1;                        // K tile landed
+  static constexpr int B_KE = B_KF + kPrefillStages;    // K tile consumed by S = Q K^T
+  static constexpr int B_VF = B_KE + kPrefillStages;    // V tile landed
+  static constexpr int B_VE = B_VF + kPrefillStages;    // V tile consumed by O += P V
+  static constexpr int B_SF = B_VE + kPrefillStages;
   static constexpr int B_SE = B_SF + 2;
   static constexpr int B_PF = B_SE + 2;
   static constexpr int B_PV = B_PF + 1;
@@ -96,7 +114,10 @@ struct FusedLayout {
   static constexpr int N_BARS = B_DEC + kFusedWarps * kFusedDecStages;
   static constexpr int MISC_OFF = BAR_OFF + N_BARS * 8;
   static constexpr int TOTAL = MISC_OFF + 64;
-  static constexpr int SMEM_BYTES = TOTAL + 1024;  // slack for 1024-byte alignment
+  // The dynamic shared memory window of a CTA without static shared memory
+  // starts 1024-byte aligned; the kernel checks it and refuses to run (status)
+  // otherwise. No slack is added: two CTAs must fit in one SM.
+  static constexpr int SMEM_BYTES = TOTAL;
 };
 
 template <int D>
@@ -109,46 +130,115 @@ struct DecodeLayout {
 };
 
 // ============================================================= LSE merge
-// One warp merges one output row of D values from n split partials, in split
-// order: M = max lse_s, w_s = exp(lse_s - M), O = sum w_s O_s / sum w_s,
-// LSE = M + ln sum w_s. Partials written by other CTAs are read with .cg.
-template <int D>
-POD_DEV void merge_row_warp(const float* po, long long po_stride, const float* pl,
-                            long long pl_stride, int n, uint16_t* out, float* lse_out, int lane) {
-  constexpr int PER = D / 32;
-  float M = -INFINITY;
-  for (int s = 0; s < n; ++s) M = fmaxf(M, __ldcg(pl + s * pl_stride));
-  float acc[PER];
+POD_DEV float warp_max(float v) {
 #pragma unroll
-  for (int i = 0; i < PER; ++i) acc[i] = 0.f;
-  float W = 0.f;
-  for (int s = 0; s < n; ++s) {
-    const float ls = __ldcg(pl + s * pl_stride);
-    const float w = (ls == -INFINITY) ? 0.f : ex2((ls - M) * kLog2e);
-    W += w;
-    const float* src = po + s * po_stride + lane * PER;
-    if constexpr (PER == 4) {
-      const float4 x = __ldcg(reinterpret_cast<const float4*>(src));
-      acc[0] = fmaf(w, x.x, acc[0]);
-      acc[1] = fmaf(w, x.y, acc[1]);
-      acc[2] = fmaf(w, x.z, acc[2]);
-      acc[3] = fmaf(w, x.w, acc[3]);
-    } else {
-      const float2 x = __ldcg(reinterpret_cast<const float2*>(src));
-      acc[0] = fmaf(w, x.x, acc[0]);
-      acc[1] = fmaf(w, x.y, acc[1]);
+  for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+  return v;
+}
+POD_DEV float warp_sum(float v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  return v;
+}
+
+// One warp merges rows i0 .. i0+RB-1 (those < nrows) of n split partials:
+// M = max_s lse_s, w_s = exp(lse_s - M), O = sum_s w_s O_s / sum_s w_s,
+// LSE = M + ln sum_s w_s. Lanes hold the splits' LSE values (32 at a time) and
+// the partial-O loads of all RB rows of a split are issued together, so the
+// merge costs a few L2 round trips per split chunk rather than per split.
+// Every output element accumulates w_s O_s in split order 0..n-1, whoever
+// calls this and with whatever RB, so all merge paths agree bitwise.
+// Partials written by other CTAs are read with ld.global.cg (L2, not L1).
+template <int D, int RB>
+POD_DEV void merge_rows_warp(const float* po, long long po_split, long long po_row,
+                             const float* pl, long long pl_split, long long pl_row, int n, int i0,
+                             int nrows, uint16_t* out, long long out_row, float* lse_out,
+                             long long lse_row, int lane) {
+  constexpr int PER = D / 32;
+  float M[RB], W[RB], acc[RB][PER];
+#pragma unroll
+  for (int rb = 0; rb < RB; ++rb) {
+    M[rb] = -INFINITY;
+    W[rb] = 0.f;
+#pragma unroll
+    for (int k = 0; k < PER; ++k) acc[rb][k] = 0.f;
+  }
+  for (int s0 = 0; s0 < n; s0 += 32) {
+    const int s = s0 + lane;
+#pragma unroll
+    for (int rb = 0; rb < RB; ++rb) {
+      const float v = (s < n && i0 + rb < nrows) ? __ldcg(pl + s * pl_split + (i0 + rb) * pl_row)
+                                                 : -INFINITY;
+      M[rb] = fmaxf(M[rb], v);
     }
   }
-  const float inv = 1.f / W;
-  if constexpr (PER == 4) {
-    uint2 v;
-    v.x = pack_bf16(acc[0] * inv, acc[1] * inv);
-    v.y = pack_bf16(acc[2] * inv, acc[3] * inv);
-    *reinterpret_cast<uint2*>(out + lane * 4) = v;
-  } else {
-    *reinterpret_cast<uint32_t*>(out + lane * 2) = pack_bf16(acc[0] * inv, acc[1] * inv);
+#pragma unroll
+  for (int rb = 0; rb < RB; ++rb) M[rb] = warp_max(M[rb]);
+  for (int s0 = 0; s0 < n; s0 += 32) {
+    const int s = s0 + lane;
+    float w[RB];
+#pragma unroll
+    for (int rb = 0; rb < RB; ++rb) {
+      const float v = (s < n && i0 + rb < nrows) ? __ldcg(pl + s * pl_split + (i0 + rb) * pl_row)
+                                                 : -INFINITY;
+      w[rb] = (v == -INFINITY) ? 0.f : ex2((v - M[rb]) * kLog2e);
+      W[rb] += w[rb];
+    }
+    const int cnt = min(32, n - s0);
+#pragma unroll 2
+    for (int t = 0; t < cnt; ++t) {
+      const float* src = po + (long long)(s0 + t) * po_split + lane * PER;
+      float x[RB][PER];
+#pragma unroll
+      for (int rb = 0; rb < RB; ++rb) {
+        if (i0 + rb < nrows) {
+          if constexpr (PER == 4) {
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(src + (i0 + rb) * po_row));
+            x[rb][0] = v.x; x[rb][1] = v.y; x[rb][2] = v.z; x[rb][3] = v.w;
+          } else {
+            const float2 v = __ldcg(reinterpret_cast<const float2*>(src + (i0 + rb) * po_row));
+            x[rb][0] = v.x; x[rb][1] = v.y;
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < PER; ++k) x[rb][k] = 0.f;
+        }
+      }
+#pragma unroll
+      for (int rb = 0; rb < RB; ++rb) {
+        const float wt = __shfl_sync(0xffffffffu, w[rb], t);
+#pragma unroll
+        for (int k = 0; k < PER; ++k) acc[rb][k] = fmaf(wt, x[rb][k], acc[rb][k]);
+      }
+    }
   }
-  if (lane == 0 && lse_out) *lse_out = M + logf(W);
+#pragma unroll
+  for (int rb = 0; rb < RB; ++rb) {
+    W[rb] = warp_sum(W[rb]);
+    if (i0 + rb >= nrows) continue;
+    const float inv = 1.f / W[rb];
+    uint16_t* o = out + (i0 + rb) * out_row + lane * PER;
+    if constexpr (PER == 4) {
+      uint2 v;
+      v.x = pack_bf16(acc[rb][0] * inv, acc[rb][1] * inv);
+      v.y = pack_bf16(acc[rb][2] * inv, acc[rb][3] * inv);
+      *reinterpret_cast<uint2*>(o) = v;
+    } else {
+      *reinterpret_cast<uint32_t*>(o) = pack_bf16(acc[rb][0] * inv, acc[rb][1] * inv);
+    }
+    if (lane == 0) lse_out[(i0 + rb) * lse_row] = M[rb] + logf(W[rb]);
+  }
+}
+
+// All G rows of decode merge group (request r, KV head g); one warp.
+template <int D>
+POD_DEV void merge_decode_group(const Plan& P, const DecodeReq& R, int r, int g, int lane) {
+  const int slot0 = R.slot0 + g;
+  for (int i0 = 0; i0 < P.G; i0 += 4)
+    merge_rows_warp<D, 4>(P.dpart_o + (size_t)slot0 * kMaxGroup * D, (long long)P.Hk * kMaxGroup * D,
+                          D, P.dpart_lse + (size_t)slot0 * kMaxGroup, (long long)P.Hk * kMaxGroup, 1,
+                          R.n_split, i0, P.G, P.o_d + ((size_t)r * P.H + (size_t)g * P.G) * D, D,
+                          P.lse_d + (size_t)r * P.H + (size_t)g * P.G, 1, lane);
 }
 
 // ============================================================= decode unit
@@ -237,13 +327,18 @@ POD_DEV bool decode_unit_warp(const Plan& P, int u, uint8_t* wsm, uint32_t bar0,
     const uint32_t kb = wsm_a + st * STAGE;
     const uint32_t vb = kb + kDecTile * ROW;
     // S^T[16 keys x 8 heads]
-    float c[4] = {0.f, 0.f, 0.f, 0.f};
+    // two independent accumulator chains halve the dependent mma latency
+    float c[4] = {0.f, 0.f, 0.f, 0.f}, c2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int kk = 0; kk < KS; ++kk) {
-      uint32_t a[4];
+    for (int kk = 0; kk < KS; kk += 2) {
+      uint32_t a[4], a2[4];
       ldsm_x4(kb + (lane & 15) * ROW + (kk * 16 + 8 * (lane >> 4)) * 2, a);
+      ldsm_x4(kb + (lane & 15) * ROW + ((kk + 1) * 16 + 8 * (lane >> 4)) * 2, a2);
       mma_16816(c, a, qb[kk][0], qb[kk][1]);
+      mma_16816(c2, a2, qb[kk + 1][0], qb[kk + 1][1]);
     }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) c[i] += c2[i];
     const int key_a = kbeg + t * kDecTile + hrow;
     float s0 = (key_a < kend) ? c[0] * sc : -INFINITY;
     float s1 = (key_a < kend) ? c[1] * sc : -INFINITY;
@@ -362,13 +457,7 @@ POD_DEV bool decode_unit_warp(const Plan& P, int u, uint8_t* wsm, uint32_t bar0,
   last = __shfl_sync(0xffffffffu, last, 0);
   if (!last) return true;
   __threadfence();
-  for (int i = 0; i < G; ++i) {
-    const int slot0 = R.slot0 + g;
-    merge_row_warp<D>(P.dpart_o + ((size_t)slot0 * kMaxGroup + i) * D, (long long)Hk * kMaxGroup * D,
-                      P.dpart_lse + (size_t)slot0 * kMaxGroup + i, (long long)Hk * kMaxGroup,
-                      R.n_split, P.o_d + ((size_t)r * P.H + (size_t)g * G + i) * D,
-                      P.lse_d + (size_t)r * P.H + (size_t)g * G + i, lane);
-  }
+  merge_decode_group<D>(P, R, r, g, lane);
   return true;
 }
 
@@ -395,13 +484,15 @@ POD_DEV PrefillRange prefill_range(const Plan& P, int u) {
 
 // Per-CTA iteration counters that carry mbarrier phases across units.
 struct PipeState {
-  uint32_t kv;  // KV tiles processed
-  uint32_t q;   // Q tiles loaded
-  uint32_t s;   // S tiles (= kv)
-  uint32_t pv;  // PV completions observed by softmax threads
+  uint32_t kv;       // KV tiles processed
+  uint32_t q;        // Q tiles loaded
+  uint32_t pv;       // PV completions observed by softmax threads
+  uint32_t kissued;  // producer: K tiles issued (for the abort drain)
+  uint32_t vissued;  // producer: V tiles issued
 };
 
-// ---- TMA producer (one thread)
+// ---- TMA producer (one thread). Two rings: a K stage is released as soon as
+// S = Q K^T has read it, a V stage once O += P V has; K runs one tile ahead.
 template <int D>
 POD_DEV bool prefill_producer(const Plan& P, const TmaDescs& T, const PrefillRange& pr,
                               uint8_t* sm, PipeState& ps, volatile int* abort_flag) {
@@ -420,45 +511,47 @@ POD_DEV bool prefill_producer(const Plan& P, const TmaDescs& T, const PrefillRan
   const CUtensorMap* km = P.paged ? &T.k[0] : &T.k[pr.req];
   const CUtensorMap* vm = P.paged ? &T.v[0] : &T.v[pr.req];
   const int last_page = (R.kv_len - 1) >> 4;
-  for (int j = 0; j < pr.n; ++j) {
+
+  // one K or V tile of 64 keys into ring `off` stage `st`, completing on `full`
+  auto load_tile = [&](const CUtensorMap* m, uint32_t dst, uint32_t full, int key0) {
+    mbar_expect_tx(full, L::KT);
+    if (!P.paged) {
+      for (int b = 0; b < NB; ++b) tma_load_3d(dst + b * (kKVTile * 128), m, full, 64 * b, g, key0);
+    } else {
+      for (int pg = 0; pg < kKVTile / 16; ++pg) {
+        const int lp = min((key0 >> 4) + pg, last_page);
+        const int phys = __ldg(P.bt_p + (size_t)R.bt_row * P.bt_stride_p + lp);
+        for (int b = 0; b < NB; ++b)
+          tma_load_3d(dst + b * (kKVTile * 128) + pg * 16 * 128, m, full, 64 * b, g, phys * 16);
+      }
+    }
+  };
+  auto issue = [&](int j, bool is_k) -> bool {
     const uint32_t it = ps.kv + j;
     const uint32_t st = it % kPrefillStages;
     const uint32_t ph = (it / kPrefillStages) & 1;
-    if (it >= kPrefillStages) {
-      if (!wait_bar(bars + (L::B_KVE + st) * 8, ph ^ 1, P, abort_flag)) {
-        ps.kv += j;
-        return false;
-      }
+    const int empty = is_k ? L::B_KE : L::B_VE;
+    if (it >= kPrefillStages && !wait_bar(bars + (empty + st) * 8, ph ^ 1, P, abort_flag))
+      return false;
+    const uint32_t dst = base + (is_k ? L::K_OFF : L::V_OFF) + st * L::KT;
+    load_tile(is_k ? km : vm, dst, bars + ((is_k ? L::B_KF : L::B_VF) + st) * 8,
+              (pr.t0 + j) * kKVTile);
+    return true;
+  };
+  bool ok = issue(0, true);
+  ps.kissued = ps.kv + 1;
+  for (int j = 0; ok && j < pr.n; ++j) {
+    if (j + 1 < pr.n) {
+      ok = issue(j + 1, true);
+      if (ok) ps.kissued = ps.kv + j + 2;
     }
-    const int key0 = (pr.t0 + j) * kKVTile;
-    const uint32_t kdst = base + L::K_OFF + st * L::KT;
-    const uint32_t vdst = base + L::V_OFF + st * L::KT;
-    const uint32_t kf = bars + (L::B_KF + st) * 8, vf = bars + (L::B_VF + st) * 8;
-    mbar_expect_tx(kf, L::KT);
-    if (!P.paged) {
-      for (int b = 0; b < NB; ++b) tma_load_3d(kdst + b * (kKVTile * 128), km, kf, 64 * b, g, key0);
-    } else {
-      for (int pg = 0; pg < kKVTile / 16; ++pg) {
-        const int lp = min((key0 >> 4) + pg, last_page);
-        const int phys = __ldg(P.bt_p + (size_t)R.bt_row * P.bt_stride_p + lp);
-        for (int b = 0; b < NB; ++b)
-          tma_load_3d(kdst + b * (kKVTile * 128) + pg * 16 * 128, km, kf, 64 * b, g, phys * 16);
-      }
-    }
-    mbar_expect_tx(vf, L::KT);
-    if (!P.paged) {
-      for (int b = 0; b < NB; ++b) tma_load_3d(vdst + b * (kKVTile * 128), vm, vf, 64 * b, g, key0);
-    } else {
-      for (int pg = 0; pg < kKVTile / 16; ++pg) {
-        const int lp = min((key0 >> 4) + pg, last_page);
-        const int phys = __ldg(P.bt_p + (size_t)R.bt_row * P.bt_stride_p + lp);
-        for (int b = 0; b < NB; ++b)
-          tma_load_3d(vdst + b * (kKVTile * 128) + pg * 16 * 128, vm, vf, 64 * b, g, phys * 16);
-      }
+    if (ok) {
+      ok = issue(j, false);
+      if (ok) ps.vissued = ps.kv + j + 1;
     }
   }
   ps.kv += pr.n;
-  return true;
+  return ok;
 }
 
 template <int D>
@@ -466,11 +559,15 @@ POD_DEV void prefill_producer_drain(const Plan& P, uint8_t* sm, const PipeState&
   using L = FusedLayout<D>;
   const uint32_t bars = smem_u32(sm) + L::BAR_OFF;
   if (ps.q > 0) drain_bar(bars + L::B_Q * 8, (ps.q - 1) & 1, P.wait_budget);
-  for (uint32_t k = 0; k < kPrefillStages && k < ps.kv; ++k) {
-    const uint32_t it = ps.kv - 1 - k;
-    const uint32_t st = it % kPrefillStages, ph = (it / kPrefillStages) & 1;
-    drain_bar(bars + (L::B_KF + st) * 8, ph, P.wait_budget);
-    drain_bar(bars + (L::B_VF + st) * 8, ph, P.wait_budget);
+  for (uint32_t k = 0; k < kPrefillStages && k < ps.kissued; ++k) {
+    const uint32_t it = ps.kissued - 1 - k;
+    drain_bar(bars + (L::B_KF + it % kPrefillStages) * 8, (it / kPrefillStages) & 1,
+              P.wait_budget);
+  }
+  for (uint32_t k = 0; k < kPrefillStages && k < ps.vissued; ++k) {
+    const uint32_t it = ps.vissued - 1 - k;
+    drain_bar(bars + (L::B_VF + it % kPrefillStages) * 8, (it / kPrefillStages) & 1,
+              P.wait_budget);
   }
 }
 
@@ -495,7 +592,7 @@ POD_DEV bool prefill_mma(const Plan& P, const PrefillRange& pr, uint8_t* sm, uin
     if (!wait_bar(bars + L::B_PF * 8, it & 1, P, abort_flag)) return false;
     if (!wait_bar(bars + (L::B_VF + st) * 8, ph, P, abort_flag)) return false;
     tc_fence_after();
-    const uint32_t pbase = (D >= 128) ? (base + L::K_OFF + st * L::KT) : (base + L::P_OFF);
+    const uint32_t pbase = base + L::P_OFF;
     const uint32_t vbase = base + L::V_OFF + st * L::KT;
 #pragma unroll
     for (int kk = 0; kk < kKVTile / 16; ++kk) {
@@ -504,7 +601,7 @@ POD_DEV bool prefill_mma(const Plan& P, const PrefillRange& pr, uint8_t* sm, uin
       umma_ss(tmem + 0, ad, bd, IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
     }
     umma_commit(bars + L::B_PV * 8);
-    umma_commit(bars + (L::B_KVE + st) * 8);
+    umma_commit(bars + (L::B_VE + st) * 8);
     last_commit_bar = bars + L::B_PV * 8;
     last_commit_par = it & 1;  // pv_done completes once per tile
     return true;
@@ -527,6 +624,7 @@ POD_DEV bool prefill_mma(const Plan& P, const PrefillRange& pr, uint8_t* sm, uin
       umma_ss(tmem + 128 + 64 * b, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
     }
     umma_commit(bars + (L::B_SF + b) * 8);
+    umma_commit(bars + (L::B_KE + st) * 8);  // K stage free once S has read it
     last_commit_bar = bars + (L::B_SF + b) * 8;
     last_commit_par = (it >> 1) & 1;
     if (j > 0 && !issue_pv(j - 1)) return false;
@@ -556,7 +654,6 @@ POD_DEV bool prefill_softmax(const Plan& P, const PrefillRange& pr, uint8_t* sm,
 
   for (int j = 0; j < pr.n; ++j) {
     const uint32_t it = ps.kv + j;
-    const uint32_t st = it % kPrefillStages;
     const uint32_t b = it & 1;
     if (!wait_bar_warp(bars + (L::B_SF + b) * 8, (it >> 1) & 1, P, abort_flag)) {
       failed = true;
@@ -564,8 +661,7 @@ POD_DEV bool prefill_softmax(const Plan& P, const PrefillRange& pr, uint8_t* sm,
     }
     tc_fence_after();
     uint32_t sr[2][32];
-    tmem_ld32(tmem + lane_base + 128 + 64 * b, sr[0]);
-    tmem_ld32(tmem + lane_base + 128 + 64 * b + 32, sr[1]);
+    tmem_ld32x2(tmem + lane_base + 128 + 64 * b, sr[0], sr[1]);
     tc_fence_before();
     mbar_arrive(bars + (L::B_SE + b) * 8);
 
@@ -573,15 +669,23 @@ POD_DEV bool prefill_softmax(const Plan& P, const PrefillRange& pr, uint8_t* sm,
     float s[64];
 #pragma unroll
     for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(sr[c >> 5][c & 31]);
-    if (key0 + kKVTile - 1 > mask_from) {
+    const bool masked_tile = key0 + kKVTile - 1 > mask_from;  // uniform over the CTA
+    if (masked_tile) {
 #pragma unroll
       for (int c = 0; c < 64; ++c)
         if (key0 + c > lim) s[c] = -INFINITY;
     }
-    float mx = -INFINITY;
+    float mx;
+    {
+      float t[32];
 #pragma unroll
-    for (int c = 0; c < 64; ++c) mx = fmaxf(mx, s[c]);
-    mx *= sc;
+      for (int c = 0; c < 32; ++c) t[c] = fmaxf(s[c], s[c + 32]);
+#pragma unroll
+      for (int w = 16; w >= 1; w >>= 1)
+#pragma unroll
+        for (int c = 0; c < w; ++c) t[c] = fmaxf(t[c], t[c + w]);
+      mx = t[0] * sc;
+    }
     // Lazy rescale: keep the reference max unless the tile max exceeds it by
     // more than 8 (log2 units), which bounds P by 2^8.
     float alpha = 1.f;
@@ -593,17 +697,38 @@ POD_DEV bool prefill_softmax(const Plan& P, const PrefillRange& pr, uint8_t* sm,
     }
     const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
     uint32_t pk[32];
-    float lt = 0.f;
+    float lt;
+    {
+      float t[32];
+      if (masked_tile) {
 #pragma unroll
-    for (int c = 0; c < 32; ++c) {
-      const float p0 = ex2(fmaf(s[2 * c], sc, -m_use));
-      const float p1 = ex2(fmaf(s[2 * c + 1], sc, -m_use));
-      pk[c] = pack_bf16(p0, p1);
-      lt += p0 + p1;  // unrounded weights (see the decode path)
+        for (int c = 0; c < 32; ++c) {
+          const float p0 = ex2(fmaf(s[2 * c], sc, -m_use));
+          const float p1 = ex2(fmaf(s[2 * c + 1], sc, -m_use));
+          pk[c] = POD_PACK(p0, p1);
+          t[c] = p0 + p1;  // unrounded weights (see the decode path)
+        }
+      } else {
+        // kSoftPairs of every 8 column pairs on the FMA pipe, the rest on MUFU
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const float x0 = fmaf(s[2 * c], sc, -m_use), x1 = fmaf(s[2 * c + 1], sc, -m_use);
+          const bool soft = (c & 7) >= 8 - kSoftPairs;
+          const float p0 = soft ? exp2_poly(x0) : ex2(x0);
+          const float p1 = soft ? exp2_poly(x1) : ex2(x1);
+          pk[c] = POD_PACK(p0, p1);
+          t[c] = p0 + p1;
+        }
+      }
+#pragma unroll
+      for (int w = 16; w >= 1; w >>= 1)
+#pragma unroll
+        for (int c = 0; c < w; ++c) t[c] += t[c + w];
+      lt = t[0];
     }
     l_run = l_run * alpha + lt;
-    // PV of the previous tile must be done before O is touched (and before
-    // the separate P buffer is overwritten when d < 128).
+    // PV of the previous tile must be done before O is touched and before
+    // the P buffer is overwritten.
     if (j > 0) {
       if (!wait_bar_warp(bars + L::B_PV * 8, ps.pv & 1, P, abort_flag)) {
         failed = true;
@@ -626,7 +751,7 @@ POD_DEV bool prefill_softmax(const Plan& P, const PrefillRange& pr, uint8_t* sm,
       }
     }
     // P (bf16, 128 rows x 64 keys, K-major, 128-byte swizzle) into smem.
-    uint8_t* prow = sm + ((D >= 128) ? (L::K_OFF + st * L::KT) : L::P_OFF) + row * 128;
+    uint8_t* prow = sm + L::P_OFF + row * 128;
 #pragma unroll
     for (int ch = 0; ch < 8; ++ch) {
       uint4 v = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
@@ -706,13 +831,13 @@ POD_DEV bool prefill_softmax(const Plan& P, const PrefillRange& pr, uint8_t* sm,
     __threadfence();
     const int rows = min(kQTile, RR.chunk - pr.qtile * kQTile);
     const int slot0 = RR.slot0 + gidx * RR.n_split;
-    for (int rr = warp; rr < rows; rr += 4) {
-      const size_t orow = (size_t)(RR.q_row0 + pr.qtile * kQTile + rr);
-      merge_row_warp<D>(P.ppart_o + ((size_t)slot0 * kQTile + rr) * D, (long long)kQTile * D,
-                        P.ppart_lse + (size_t)slot0 * kQTile + rr, kQTile, RR.n_split,
-                        P.o_p + (orow * P.H + pr.head) * D, P.lse_p + orow * P.H + pr.head,
-                        tid & 31);
-    }
+    const size_t orow0 = (size_t)(RR.q_row0 + pr.qtile * kQTile);
+    // warp w merges rows [32w, 32w + 32), four at a time
+    for (int i0 = warp * 32; i0 < min(rows, warp * 32 + 32); i0 += 4)
+      merge_rows_warp<D, 4>(P.ppart_o + (size_t)slot0 * kQTile * D, (long long)kQTile * D, D,
+                            P.ppart_lse + (size_t)slot0 * kQTile, kQTile, 1, RR.n_split, i0,
+                            min(rows, warp * 32 + 32), P.o_p + (orow0 * P.H + pr.head) * D,
+                            (long long)P.H * D, P.lse_p + orow0 * P.H + pr.head, P.H, tid & 31);
   }
   return !failed;
 }
@@ -725,10 +850,13 @@ __global__ void __launch_bounds__(kFusedThreads, kFusedSlotsPerSm)
     pod_fused_kernel(const __grid_constant__ Plan P, const __grid_constant__ TmaDescs T,
                      int allow_prefill, int allow_decode) {
   using L = FusedLayout<D>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                           ~(uintptr_t)1023);
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* sm = smem_raw;
   const int tid = threadIdx.x;
+  if (smem_u32(sm) & 1023u) {  // 128-byte swizzle atoms need 1024-byte alignment
+    if (tid == 0) set_status(P, kStatusUnsupported);
+    return;
+  }
   const int warp = tid >> 5, lane = tid & 31;
   const uint32_t bars = smem_u32(sm) + L::BAR_OFF;
   int* misc = reinterpret_cast<int*>(sm + L::MISC_OFF);
@@ -769,7 +897,7 @@ __global__ void __launch_bounds__(kFusedThreads, kFusedSlotsPerSm)
   }
 
   const uint32_t my_sm = smid() & (kMaxSmid - 1);
-  PipeState ps = {0u, 0u, 0u, 0u};
+  PipeState ps = {0u, 0u, 0u, 0u, 0u};
   uint32_t dec_ring = 0;
   uint32_t last_commit_bar = 0, last_commit_par = 0;
   bool issued_mma = false;
@@ -849,16 +977,15 @@ __global__ void __launch_bounds__(kFusedThreads, kFusedSlotsPerSm)
 }
 
 // ============================================================= decode-only kernels
+// Persistent: every warp is a virtual decode unit runner that claims the next
+// unit from the decode queue until it is empty.
 template <int D>
 __global__ void __launch_bounds__(kDecodeWarps * 32)
     pod_decode_kernel(const __grid_constant__ Plan P) {
   using L = DecodeLayout<D>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 15) &
-                                           ~(uintptr_t)15);
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* sm = smem_raw;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int u = blockIdx.x * kDecodeWarps + warp;
-  if (u >= P.n_decode_units) return;
   const uint32_t bar0 = smem_u32(sm + L::BAR_OFF) + warp * kDecodeStages * 8;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::BAR_OFF +
                                                               kDecodeWarps * kDecodeStages * 8) +
@@ -870,24 +997,27 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
   }
   __syncwarp();
   uint32_t ring = 0;
-  decode_unit_warp<D, kDecodeStages>(P, u, sm + warp * L::WARP, bar0, ring, lane, false, abort_flag);
+  while (true) {
+    int u = 0;
+    if (lane == 0) u = atomicAdd(P.ctl + 1, 1);
+    u = __shfl_sync(0xffffffffu, u, 0);
+    if (u >= P.n_decode_units) break;
+    if (!decode_unit_warp<D, kDecodeStages>(P, u, sm + warp * L::WARP, bar0, ring, lane, false,
+                                            abort_flag))
+      break;
+  }
 }
 
-// One warp per (decode request, query head) whose KV range was split.
+// One warp per (decode request, KV head) group whose KV range was split.
 template <int D>
 __global__ void __launch_bounds__(128) pod_merge_kernel(const __grid_constant__ Plan P) {
   const int gw = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (gw >= P.n_decode_reqs * P.H) return;
-  const int r = gw / P.H, h = gw - (gw / P.H) * P.H;
+  if (gw >= P.n_decode_reqs * P.Hk) return;
+  const int r = gw / P.Hk, g = gw - (gw / P.Hk) * P.Hk;
   const DecodeReq R = P.dreq[r];
   if (R.n_split <= 1) return;
-  const int g = h / P.G, i = h - (h / P.G) * P.G;
-  const int slot0 = R.slot0 + g;
-  merge_row_warp<D>(P.dpart_o + ((size_t)slot0 * kMaxGroup + i) * D,
-                    (long long)P.Hk * kMaxGroup * D, P.dpart_lse + (size_t)slot0 * kMaxGroup + i,
-                    (long long)P.Hk * kMaxGroup, R.n_split, P.o_d + ((size_t)r * P.H + h) * D,
-                    P.lse_d + (size_t)r * P.H + h, lane);
+  merge_decode_group<D>(P, R, r, g, lane);
 }
 
 // ============================================================= host-side launchers
@@ -921,8 +1051,19 @@ cudaError_t launch_fused(const Plan& P, const TmaDescs& T, int grid, int allow_p
   return cudaGetLastError();
 }
 
-cudaError_t launch_decode(const Plan& P, cudaStream_t s) {
-  const int grid = (P.n_decode_units + kDecodeWarps - 1) / kDecodeWarps;
+cudaError_t decode_occupancy(int D, int* blocks_per_sm) {
+  if (D == 128)
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pod_decode_kernel<128>,
+                                                         kDecodeWarps * 32,
+                                                         DecodeLayout<128>::SMEM_BYTES);
+  return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, pod_decode_kernel<64>,
+                                                       kDecodeWarps * 32,
+                                                       DecodeLayout<64>::SMEM_BYTES);
+}
+
+cudaError_t launch_decode(const Plan& P, int max_grid, cudaStream_t s) {
+  const int need = (P.n_decode_units + kDecodeWarps - 1) / kDecodeWarps;
+  const int grid = need < max_grid ? need : max_grid;
   if (grid == 0) return cudaSuccess;
   if (P.D == 128)
     pod_decode_kernel<128><<<grid, kDecodeWarps * 32, DecodeLayout<128>::SMEM_BYTES, s>>>(P);
@@ -932,7 +1073,7 @@ cudaError_t launch_decode(const Plan& P, cudaStream_t s) {
 }
 
 cudaError_t launch_merge(const Plan& P, cudaStream_t s) {
-  const int rows = P.n_decode_reqs * P.H;
+  const int rows = P.n_decode_reqs * P.Hk;
   const int grid = (rows + 3) / 4;
   if (grid == 0) return cudaSuccess;
   if (P.D == 128)

@@ -23,8 +23,8 @@ constexpr int kFusedWarps = 6;        // 4 softmax + 1 MMA issuer + 1 TMA produc
 constexpr int kFusedThreads = kFusedWarps * 32;
 constexpr int kFusedSlotsPerSm = 2;   // persistent CTAs per SM
 constexpr int kFusedDecStages = 2;    // per-warp decode ring depth in the fused kernel
-constexpr int kDecodeWarps = 4;       // warps (virtual decode units) per decode-only CTA
-constexpr int kDecodeStages = 3;      // per-warp ring depth in the decode-only kernel
+constexpr int kDecodeWarps = 6;       // warps (virtual decode units) per decode-only CTA
+constexpr int kDecodeStages = 2;      // per-warp ring depth in the decode-only kernel
 constexpr int kMaxGroup = 8;          // query heads per KV head (mma N = 8)
 constexpr int kTmemCols = 256;        // TMEM columns per CTA: O [0,128), S0, S1 [128,256)
 constexpr int kMaxSmid = 256;         // per-SM ticket slots (indexed by %smid)

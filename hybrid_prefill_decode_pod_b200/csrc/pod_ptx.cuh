@@ -126,6 +126,8 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N, int a_mn_ma
 
 #define POD_R8(i) "=r"(r[i]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), \
                   "=r"(r[i + 4]), "=r"(r[i + 5]), "=r"(r[i + 6]), "=r"(r[i + 7])
+#define POD_R8B(i) "=r"(r2[i]), "=r"(r2[i + 1]), "=r"(r2[i + 2]), "=r"(r2[i + 3]), \
+                   "=r"(r2[i + 4]), "=r"(r2[i + 5]), "=r"(r2[i + 6]), "=r"(r2[i + 7])
 #define POD_W8(i) "r"(r[i]), "r"(r[i + 1]), "r"(r[i + 2]), "r"(r[i + 3]), \
                   "r"(r[i + 4]), "r"(r[i + 5]), "r"(r[i + 6]), "r"(r[i + 7])
 
@@ -139,6 +141,21 @@ POD_DEV void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       "tcgen05.wait::ld.sync.aligned;"
       : POD_R8(0), POD_R8(8), POD_R8(16), POD_R8(24)
       : "r"(taddr)
+      : "memory");
+}
+// 64 consecutive columns in two x32 loads under one wait.
+POD_DEV void tmem_ld32x2(uint32_t taddr, uint32_t (&r)[32], uint32_t (&r2)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%64];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : POD_R8(0), POD_R8(8), POD_R8(16), POD_R8(24), POD_R8B(0), POD_R8B(8), POD_R8B(16),
+        POD_R8B(24)
+      : "r"(taddr), "r"(taddr + 32)
       : "memory");
 }
 POD_DEV void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
@@ -182,6 +199,14 @@ POD_DEV uint32_t pack_bf16(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+// Same rounding (nearest even) with integer ops only, for finite inputs: keeps
+// the conversion off the XU pipe that ex2 uses.
+POD_DEV uint32_t pack_bf16_int(float lo, float hi) {
+  uint32_t a = __float_as_uint(lo), b = __float_as_uint(hi);
+  a += 0x7FFFu + ((a >> 16) & 1u);
+  b += 0x7FFFu + ((b >> 16) & 1u);
+  return __byte_perm(a, b, 0x7632);
 }
 POD_DEV float bf16_lo(uint32_t x) { return __uint_as_float(x << 16); }
 POD_DEV float bf16_hi(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }

@@ -78,6 +78,13 @@ CONFIGS = {
         decode_range=(1024, 16384, 128), paged=True),
 }
 
+# Smaller batches of the same shape families, for profiler captures (a capture
+# replays each launch many times, so it is taken on a reduced case).
+PROBE_CONFIGS = {
+    "long_context_probe": HybridConfig(
+        "long_context_probe", 64, 8, 128, prefill=((4096, 1024),), decode_ctx=(4096,) * 16),
+}
+
 # Human-readable descriptions used in the benchmark's JSON line.
 CONFIG_DESCRIPTIONS = {
     "tiny": "tiny hybrid batch: 1 prefill (prior 64 + chunk 32) + 4 decodes (40/77/128/200), 4 q / 2 kv heads, d 64",
@@ -85,7 +92,12 @@ CONFIG_DESCRIPTIONS = {
     "decode_heavy": "decode-heavy: 32 q / 8 kv heads, d 128; 1 prefill chunk 256 after prior 1024 + 256 decodes U[512, 8192]",
     "long_context": "long-context 70B-like: 64 q / 8 kv heads, d 128; 1 prefill chunk 1024 after prior 16384 + 16 decodes U[16384, 32768]",
     "paged": "paged-KV: 32 q / 8 kv heads, d 128; 2 prefill chunks of 512 (priors 2048, 8192) + 128 decodes U[1024, 16384], 16-token blocks, permuted",
+    "long_context_probe": "profiling probe: 64 q / 8 kv heads, d 128; 1 prefill chunk 1024 after prior 4096 + 16 decodes at 4096",
 }
+
+
+def get_config(name: str) -> HybridConfig:
+    return CONFIGS[name] if name in CONFIGS else PROBE_CONFIGS[name]
 
 
 @dataclasses.dataclass

@@ -98,7 +98,9 @@ def test_invariants_on_gpu():
     for r, L in enumerate(b.ctx):
         assert np.abs(out["decode_lse"][r].numpy() - np.log(L)).max() < 1e-5
     t = np.arange(150)
-    assert np.abs(out["prefill_lse"].numpy() - np.log(t + 1)[:, None]).max() < 1e-5
+    # prefill evaluates 3/8 of its exponentials with a polynomial whose relative
+    # error is below 7.5e-5 (csrc/pod_exp2.cuh), which bounds the LSE error here
+    assert np.abs(out["prefill_lse"].numpy() - np.log(t + 1)[:, None]).max() < 1e-4
     # single key: decode L = 1 returns V0 bitwise
     b2 = W.make_custom(8, 2, 128, [], [1, 1], seed=23)
     out2, _ = run(b2, "fused")
