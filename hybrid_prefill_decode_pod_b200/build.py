@@ -14,7 +14,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libpod_attn.so")
-SOURCES = [os.path.join(CSRC, "pod_kernels.cu"), os.path.join(CSRC, "pod_attn_api.cpp")]
+SOURCES = [os.path.join(CSRC, "pod_kernels.cu"), os.path.join(CSRC, "pod_attn_api.cpp"),
+           os.path.join(CSRC, "pod_static.cu")]
 HEADERS = [os.path.join(CSRC, f) for f in ("pod_plan.h", "pod_ptx.cuh", "pod_exp2.cuh")] + [
     os.path.join(INCLUDE, "pod_attn.h")]
 

@@ -41,7 +41,8 @@ FLAG_TEST_FORCE_TIMEOUT = 0x2
 # Every symbol include/pod_attn.h declares.
 EXPORTED = ("pod_attn_create", "pod_attn_hybrid", "pod_attn_prefill_only",
             "pod_attn_decode_only", "pod_attn_status", "pod_attn_last_plan",
-            "pod_attn_get_stats", "pod_attn_destroy", "pod_attn_strerror")
+            "pod_attn_get_stats", "pod_attn_destroy", "pod_attn_decode_static",
+            "pod_attn_strerror")
 
 
 class PodError(RuntimeError):
@@ -118,6 +119,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pod_attn_last_plan.argtypes = [vp, ctypes.POINTER(PlanInfo)]
     lib.pod_attn_get_stats.argtypes = [vp, vp, ctypes.POINTER(Stats)]
     lib.pod_attn_destroy.argtypes = [vp]
+    lib.pod_attn_decode_static.argtypes = [i, i, i, i, ctypes.POINTER(DecodeArgs), vp]
     lib.pod_attn_strerror.argtypes = [i]
     lib.pod_attn_strerror.restype = ctypes.c_char_p
     for name in EXPORTED:
@@ -280,6 +282,19 @@ class PodAttention:
             self.close()
         except Exception:
             pass
+
+
+def decode_static(num_qo_heads: int, num_kv_heads: int, head_dim: int, decode: DecodeArgs,
+                  paged: bool = False, stream=None) -> None:
+    """``pod_attn_decode_static``: decode attention that allocates no device
+    memory (for callers whose device memory is all owned by someone else).
+    Runs on the current CUDA device; calls must not overlap on the GPU."""
+    lib = load_library()
+    rc = lib.pod_attn_decode_static(int(num_qo_heads), int(num_kv_heads), int(head_dim),
+                                    POD_KV_PAGED if paged else POD_KV_CONTIGUOUS,
+                                    ctypes.byref(decode), ctypes.c_void_p(_stream_handle(stream)))
+    if rc != POD_OK:
+        raise PodError(rc, "pod_attn_decode_static")
 
 
 class DeviceBatch:

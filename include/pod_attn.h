@@ -203,6 +203,47 @@ POD_API int pod_attn_get_stats(pod_attn_ctx* ctx, void* stream, pod_stats* out);
  * Returns that status (POD_OK or POD_ETIMEOUT) or POD_ECUDA. NULL is a no-op. */
 POD_API int pod_attn_destroy(pod_attn_ctx* ctx);
 
+/* ---------------------------------------------------------------------------
+ * Decode attention that allocates nothing (no counterpart in the paper: it
+ * is a deployment convenience of this library).
+ *
+ * For callers that cannot allocate device memory when they call attention:
+ * an inference engine that reserves nearly all HBM for its KV-cache pool up
+ * front, a plugin that may only use the buffers its host framework gives it,
+ * or a loop that cannot afford cudaMalloc's implicit synchronisation. A
+ * pod_attn context allocates its workspace at create time, so this entry
+ * point needs none: it runs the same split-KV decode and LSE merge kernels as
+ * pod_attn_decode_only, with their plan tables, counters and partial results
+ * in a fixed device array inside the library (about 16.5 MB, present on
+ * every GPU that loads the library until the process exits). It calls no
+ * cudaMalloc, cudaFree or other allocating routine.
+ *
+ * Arguments: head counts and head_dim as in pod_attn_config, kv_layout a
+ * pod_kv_layout, `args` exactly as for pod_attn_decode_only (caller-owned
+ * device tensors, host length and pointer arrays), `stream` a cudaStream_t.
+ * The call runs on the calling thread's current device.
+ *
+ * Limits (POD_ECAPACITY beyond them, checked before anything is enqueued):
+ * num_reqs <= POD_STATIC_MAX_DECODE_REQS, num_kv_heads <=
+ * POD_STATIC_MAX_KV_HEADS, num_reqs * num_kv_heads <= POD_STATIC_MAX_UNITS.
+ * Other errors as for pod_attn_decode_only.
+ *
+ * The first call on a device resolves the array's device address and sets
+ * the kernels' shared-memory limits for that device; make that first call
+ * before any stream capture. Every call reuses the same array and leaves its
+ * contents behind (each call re-initialises what must start at zero), so
+ * calls that overlap on the GPU -- on different streams or from different
+ * host threads -- race on it and must not be issued. The copy of the small
+ * per-call plan comes from pageable host memory, so the call does not return
+ * before the stream has reached it. A device-side wait that runs out is not
+ * reported by this entry point (it has no context to hold a status word).
+ * ------------------------------------------------------------------------- */
+#define POD_STATIC_MAX_DECODE_REQS 512
+#define POD_STATIC_MAX_KV_HEADS 16
+#define POD_STATIC_MAX_UNITS 4096
+POD_API int pod_attn_decode_static(int num_qo_heads, int num_kv_heads, int head_dim,
+                                   int kv_layout, const pod_decode_args* args, void* stream);
+
 /* Static string for a pod_status value. */
 POD_API const char* pod_attn_strerror(int status);
 
