@@ -40,7 +40,6 @@ namespace {
 
 constexpr int kRing = 8;            // pinned host plan slots
 constexpr int kMaxPrefillSplit = 16;
-constexpr int kDecSplitMin = 512;   // keys per decode split, smallest
 constexpr int kDecSplitMax = 1 << 20;
 constexpr int kStatsInts = kMaxSmid * 2;
 
@@ -71,6 +70,12 @@ struct pod_attn_ctx {
   pod_attn_config cfg{};
   int device = 0, num_sms = 0, slots_per_sm = kFusedSlotsPerSm;
   int decode_grid = 0;  // persistent decode-only grid (SMs x resident CTAs)
+  // scheduling levers (defaults; environment overrides exist for ablations)
+  int policy = 4;        // 0 proportional, 1 even (50:50), 2 prefill first, 3 decode first,
+                         // 4 front (each SM's first tickets take prefill, then 50:50)
+  int smid_aware = 1;    // per-SM tickets (1) or one global ticket counter (0)
+  int dec_turn = 1;      // decode units each warp claims per decode turn of a fused CTA
+  int dec_split = 0;     // 0: cost model; else keys per decode split (multiple of 16)
   int H = 0, Hk = 0, G = 0, D = 0;
   int cap_punits = 0, cap_pgroups = 0, cap_pslots = 0;
   int cap_dunits = 0, cap_dgroups = 0, cap_dslots = 0, cap_dreqs = 0;
@@ -234,9 +239,10 @@ int build_plan(pod_attn_ctx* c, const pod_prefill_args* pa, const pod_decode_arg
       R.n_split = 1;
       continue;
     }
-    // smallest tile's KV range, in 64-key tiles; keep >= 4 tiles per split
+    // smallest tile's KV range, in 64-key tiles; a split keeps >= 16 tiles so
+    // its fixed costs (Q load, pipeline fill, partial write, merge) stay small
     const int min_tiles = (prior + std::min(chunk, kQTile) + kKVTile - 1) / kKVTile;
-    int split = std::min(split_base, std::max(1, min_tiles / 4));
+    int split = std::min(split_base, std::max(1, min_tiles / 16));
     split = std::min(split, kMaxPrefillSplit);
     R.n_split = split;
     R.n_kvtiles_max = (prior + chunk + kKVTile - 1) / kKVTile;
@@ -271,20 +277,46 @@ int build_plan(pod_attn_ctx* c, const pod_prefill_args* pa, const pod_decode_arg
   // ---- decode
   DecodeReq* dreq = reinterpret_cast<DecodeReq*>(h + L.dreq);
   int* dunit = reinterpret_cast<int*>(h + L.dunit);
-  long long key_heads = 0;
-  for (int r = 0; r < nd; ++r) key_heads += (long long)da->ctx_lens[r] * Hk;
-  // enough units to keep every decode warp busy several times over
-  const long long target = 8LL * c->num_sms * 8;
-  int split_len = kDecSplitMin;
+  // Keys per decode split (a multiple of the 16-key decode tile): the
+  // candidate minimising an estimate of the decode makespan on the persistent
+  // decode warps. Units are claimed dynamically, so with U units of at most
+  // `mx` keys on W warps the finish time is about min(ceil(U/W) * (mx + o),
+  // sum/W + mx + o), o being a per-unit overhead (start-up, partial write,
+  // merge) of about 48 keys' worth of streaming.
   auto count_units = [&](int sl) {
     long long n = 0;
     for (int r = 0; r < nd; ++r) n += (long long)((da->ctx_lens[r] + sl - 1) / sl) * Hk;
     return n;
   };
-  while (split_len < kDecSplitMax && count_units(split_len) > std::max(target, (long long)nd * Hk))
-    split_len *= 2;
-  while (split_len < kDecSplitMax && count_units(split_len) > c->cap_dunits) split_len *= 2;
-  (void)key_heads;
+  int split_len = kDecSplitMax;
+  if (nd > 0 && c->dec_split > 0) {
+    split_len = c->dec_split;
+    while (split_len < kDecSplitMax && count_units(split_len) > c->cap_dunits) split_len *= 2;
+  } else if (nd > 0) {
+    static const int kCands[] = {256, 320, 384, 512, 640, 768, 1024, 1536, 2048, 3072, 4096,
+                                 8192, 16384, 32768, 65536, 131072, 262144, 524288, 1048576};
+    const double W = (double)std::max(1, c->decode_grid * kDecodeWarps);
+    const double o = 48.0;
+    int max_len = 1;
+    long long keys = 0;
+    for (int r = 0; r < nd; ++r) {
+      max_len = std::max(max_len, da->ctx_lens[r]);
+      keys += (long long)da->ctx_lens[r] * Hk;
+    }
+    double best = 1e300;
+    for (int sl : kCands) {
+      const long long U = count_units(sl);
+      if (U > c->cap_dunits) continue;
+      const double mx = (double)std::min(sl, max_len);
+      const double est = std::min(std::ceil((double)U / W) * (mx + o),
+                                  ((double)keys + (double)U * o) / W + mx + o);
+      if (est < best * 0.999) {
+        best = est;
+        split_len = sl;
+      }
+      if (sl >= max_len) break;  // larger splits change nothing
+    }
+  }
   int n_du = 0, n_dg = 0, n_ds = 0;
   for (int r = 0; r < nd; ++r) {
     DecodeReq& R = dreq[r];
@@ -309,8 +341,14 @@ int build_plan(pod_attn_ctx* c, const pod_prefill_args* pa, const pod_decode_arg
   if (n_dg > c->cap_dgroups || n_ds > c->cap_dslots) return POD_ECAPACITY;
 
   // ---- claim ratio (per-SM Bresenham over tickets): prefill share of claims
-  const long long dclaims = (n_du + kFusedWarps - 1) / kFusedWarps;
-  int rho_num = n_pu, rho_den = n_pu + (int)dclaims;
+  // A fused CTA's decode turn processes up to dec_turn units per warp.
+  const long long dclaims =
+      (n_du + (long long)kFusedWarps * c->dec_turn - 1) / ((long long)kFusedWarps * c->dec_turn);
+  int rho_num = n_pu, rho_den = n_pu + (int)dclaims;  // proportional (summary §5.4.2)
+  if (c->policy == 1) { rho_num = 1; rho_den = 2; }
+  if (c->policy == 2) { rho_num = 1; rho_den = 1; }
+  if (c->policy == 3) { rho_num = 0; rho_den = 1; }
+  if (c->policy == 4) { rho_num = 1; rho_den = 2; }  // front: see pod_fused_kernel
   if (rho_den == 0) rho_den = 1;
 
   // ---- kernel parameters
@@ -331,7 +369,8 @@ int build_plan(pod_attn_ctx* c, const pod_prefill_args* pa, const pod_decode_arg
   Q.paged = paged ? 1 : 0;
   Q.bt_stride_p = (np && paged) ? pa->block_table_stride : 0;
   Q.bt_stride_d = (nd && paged) ? da->block_table_stride : 0;
-  Q.flags = (int)c->cfg.flags;
+  Q.flags = (int)c->cfg.flags | (c->smid_aware ? 0 : 0x100) | (c->policy == 4 ? 0x200 : 0);
+  Q.dec_turn = c->dec_turn;
   Q.wait_budget = kDefaultWaitBudget;
   char* dp = c->d_plan;
   Q.preq = reinterpret_cast<const PrefillReq*>(dp + L.preq);
@@ -487,6 +526,18 @@ int pod_attn_create(pod_attn_ctx** out, const pod_attn_config* cfg) {
     return code;
   };
   if (kernels_init(D) != cudaSuccess) return fail(POD_ECUDA);
+  // Scheduling levers for ablations (POD-Attention §5.4): environment overrides.
+  if (const char* e = std::getenv("POD_ATTN_POLICY")) {
+    if (!std::strcmp(e, "even")) c->policy = 1;
+    else if (!std::strcmp(e, "prefill_first")) c->policy = 2;
+    else if (!std::strcmp(e, "decode_first")) c->policy = 3;
+    else if (!std::strcmp(e, "front")) c->policy = 4;
+    else if (!std::strcmp(e, "proportional")) c->policy = 0;
+  }
+  if (const char* e = std::getenv("POD_ATTN_SMID_AWARE")) c->smid_aware = std::atoi(e) != 0;
+  if (const char* e = std::getenv("POD_ATTN_DEC_TURN")) c->dec_turn = std::max(1, std::atoi(e));
+  if (const char* e = std::getenv("POD_ATTN_DEC_SPLIT"))
+    c->dec_split = std::max(0, std::atoi(e)) / kDecTile * kDecTile;
   int dec_blocks = 0;
   if (decode_occupancy(D, &dec_blocks) != cudaSuccess || dec_blocks < 1) return fail(POD_ECUDA);
   c->decode_grid = c->num_sms * dec_blocks;

@@ -38,10 +38,12 @@ namespace pod {
 #define POD_SOFT_EXP2_PAIRS 0
 #endif
 constexpr int kSoftPairs = POD_SOFT_EXP2_PAIRS;
-#ifndef POD_INT_PACK
+#if defined(POD_CVT_PACK)
 #define POD_PACK(a, b) pack_bf16(a, b)
-#else
+#elif defined(POD_INT_PACK)
 #define POD_PACK(a, b) pack_bf16_int(a, b)
+#else
+#define POD_PACK(a, b) pack_bf16_rha(a, b)
 #endif
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -676,15 +678,15 @@ POD_DEV bool prefill_softmax(const Plan& P, const PrefillRange& pr, uint8_t* sm,
         if (key0 + c > lim) s[c] = -INFINITY;
     }
     float mx;
-    {
-      float t[32];
+    {  // 64 -> 22 -> 8 -> 3 -> 1 with three-input max
+      float a[22], b8[8];
 #pragma unroll
-      for (int c = 0; c < 32; ++c) t[c] = fmaxf(s[c], s[c + 32]);
+      for (int c = 0; c < 21; ++c) a[c] = max3(s[3 * c], s[3 * c + 1], s[3 * c + 2]);
+      a[21] = s[63];
 #pragma unroll
-      for (int w = 16; w >= 1; w >>= 1)
-#pragma unroll
-        for (int c = 0; c < w; ++c) t[c] = fmaxf(t[c], t[c + w]);
-      mx = t[0] * sc;
+      for (int c = 0; c < 7; ++c) b8[c] = max3(a[3 * c], a[3 * c + 1], a[3 * c + 2]);
+      b8[7] = a[21];
+      mx = max3(max3(b8[0], b8[1], b8[2]), max3(b8[3], b8[4], b8[5]), fmaxf(b8[6], b8[7])) * sc;
     }
     // Lazy rescale: keep the reference max unless the tile max exceeds it by
     // more than 8 (log2 units), which bounds P by 2^8.
@@ -906,9 +908,13 @@ __global__ void __launch_bounds__(kFusedThreads, kFusedSlotsPerSm)
     if (tid == 0) {
       int role = 0, unit = -1;
       if (!*abort_flag) {
-        const int t = atomicAdd(P.sm_ticket + my_sm, 1);
+        // per-SM ticket (SM-aware), or one global counter when that is switched off
+        const int t = atomicAdd(P.sm_ticket + ((P.flags & 0x100) ? 0 : my_sm), 1);
         const long long num = P.rho_num, den = P.rho_den > 0 ? P.rho_den : 1;
         bool want_p = ((long long)(t + 1) * num) / den > ((long long)t * num) / den;
+        // front-loaded: each SM's first two tickets (one per resident CTA) take
+        // prefill work, so the long prefill units start first
+        if ((P.flags & 0x200) && t < kFusedSlotsPerSm) want_p = true;
         for (int attempt = 0; attempt < 2 && role == 0; ++attempt, want_p = !want_p) {
           if (want_p && !misc[5]) {
             const int u = atomicAdd(P.ctl + 0, 1);
@@ -919,13 +925,8 @@ __global__ void __launch_bounds__(kFusedThreads, kFusedSlotsPerSm)
               misc[5] = 1;
             }
           } else if (!want_p && !misc[6]) {
-            const int u = atomicAdd(P.ctl + 1, kFusedWarps);
-            if (u < P.n_decode_units) {
-              role = 2;
-              unit = u;
-            } else {
-              misc[6] = 1;
-            }
+            role = 2;  // a decode turn: the warps claim their own units
+            unit = 0;
           }
         }
         if (role && (P.flags & 0x1)) atomicAdd(P.stats + my_sm * 2 + (role - 1), 1);
@@ -952,11 +953,25 @@ __global__ void __launch_bounds__(kFusedThreads, kFusedSlotsPerSm)
         __syncwarp();
       }
     } else {
-      const int u = unit + warp;
-      if (u < P.n_decode_units) {
-        decode_unit_warp<D, kFusedDecStages>(P, u, sm + warp * L::DEC_WARP,
-                                             bars + (L::B_DEC + warp * kFusedDecStages) * 8,
-                                             dec_ring, lane, true, abort_flag);
+      // decode turn: every warp is a virtual decode unit runner and claims up
+      // to dec_turn units one at a time; once every prefill unit has been
+      // claimed there is nothing to regroup for, so the warp keeps claiming
+      // until the decode queue is empty. An empty queue ends the turn.
+      for (int k = 0;; ++k) {
+        if (k >= P.dec_turn &&
+            *reinterpret_cast<volatile const int*>(P.ctl + 0) < P.n_prefill_units)
+          break;
+        int u = 0;
+        if (lane == 0) u = atomicAdd(P.ctl + 1, 1);
+        u = __shfl_sync(0xffffffffu, u, 0);
+        if (u >= P.n_decode_units) {
+          if (lane == 0) misc[6] = 1;
+          break;
+        }
+        if (!decode_unit_warp<D, kFusedDecStages>(P, u, sm + warp * L::DEC_WARP,
+                                                  bars + (L::B_DEC + warp * kFusedDecStages) * 8,
+                                                  dec_ring, lane, true, abort_flag))
+          break;
       }
     }
     __syncthreads();

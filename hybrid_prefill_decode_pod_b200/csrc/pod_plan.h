@@ -59,6 +59,8 @@ struct Plan {
   int bt_stride_p, bt_stride_d;
   int flags;
   int pool_blocks;               // paged: blocks in the pool (bounds every block id)
+  int dec_turn;                  // decode units per warp per fused decode turn
+  int pad1;
   long long wait_budget;         // cycles a bounded wait may spin
   const PrefillReq* preq;
   const PrefillUnit* punits;
