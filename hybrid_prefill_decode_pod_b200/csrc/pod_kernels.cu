@@ -90,12 +90,10 @@ template <int D>
 struct FusedLayout {
   static constexpr int QB = kQTile * D * 2;   // Q tile bytes
   static constexpr int KT = kKVTile * D * 2;  // one K (or V) tile
-  static constexpr int PB = kQTile * kKVTile * 2;  // P tile (bf16)
   static constexpr int Q_OFF = 0;
   static constexpr int K_OFF = Q_OFF + QB;                      // K ring
   static constexpr int V_OFF = K_OFF + kPrefillStages * KT;     // V ring
-  static constexpr int P_OFF = V_OFF + kPrefillStages * KT;     // P (own buffer)
-  static constexpr int PREFILL_END = P_OFF + PB;
+  static constexpr int PREFILL_END = V_OFF + kPrefillStages * KT;
   static constexpr int DEC_ROW = D * 2 + 16;  // padded row: conflict-free ldmatrix
   static constexpr int DEC_STAGE = 2 * kDecTile * DEC_ROW;
   static constexpr int DEC_WARP = kFusedDecStages * DEC_STAGE;
@@ -109,7 +107,7 @@ struct FusedLayout {
   static constexpr int B_VF = B_KE + kPrefillStages;    // V tile landed
   static constexpr int B_VE = B_VF + kPrefillStages;    // V tile consumed by O += P V
   static constexpr int B_SF = B_VE + kPrefillStages;
-  static constexpr int B_SE = B_SF + 2;
+  static constexpr int B_SE = B_SF + 2;                 // S buffer free (its P consumed by PV)
   static constexpr int B_PF = B_SE + 2;
   static constexpr int B_PV = B_PF + 1;
   static constexpr int B_DEC = B_PV + 1;
@@ -594,16 +592,17 @@ POD_DEV bool prefill_mma(const Plan& P, const PrefillRange& pr, uint8_t* sm, uin
     if (!wait_bar(bars + L::B_PF * 8, it & 1, P, abort_flag)) return false;
     if (!wait_bar(bars + (L::B_VF + st) * 8, ph, P, abort_flag)) return false;
     tc_fence_after();
-    const uint32_t pbase = base + L::P_OFF;
     const uint32_t vbase = base + L::V_OFF + st * L::KT;
+    // P (bf16 pairs) sits in the first 32 columns of the S buffer it came from
+    const uint32_t pcol = tmem + 128 + 64 * (it & 1);
 #pragma unroll
     for (int kk = 0; kk < kKVTile / 16; ++kk) {
-      const uint64_t ad = sw128_desc(pbase + kk * 32, 16, 1024);
       const uint64_t bd = sw128_desc(vbase + kk * 16 * 128, kKVTile * 128, 1024);
-      umma_ss(tmem + 0, ad, bd, IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
+      umma_ts(tmem + 0, pcol + kk * 8, bd, IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
     }
     umma_commit(bars + L::B_PV * 8);
     umma_commit(bars + (L::B_VE + st) * 8);
+    umma_commit(bars + (L::B_SE + (it & 1)) * 8);  // S buffer free once its P is consumed
     last_commit_bar = bars + L::B_PV * 8;
     last_commit_par = it & 1;  // pv_done completes once per tile
     return true;
@@ -664,8 +663,6 @@ POD_DEV bool prefill_softmax(const Plan& P, const PrefillRange& pr, uint8_t* sm,
     tc_fence_after();
     uint32_t sr[2][32];
     tmem_ld32x2(tmem + lane_base + 128 + 64 * b, sr[0], sr[1]);
-    tc_fence_before();
-    mbar_arrive(bars + (L::B_SE + b) * 8);
 
     const int key0 = (pr.t0 + j) * kKVTile;
     float s[64];
@@ -688,49 +685,47 @@ POD_DEV bool prefill_softmax(const Plan& P, const PrefillRange& pr, uint8_t* sm,
       b8[7] = a[21];
       mx = max3(max3(b8[0], b8[1], b8[2]), max3(b8[3], b8[4], b8[5]), fmaxf(b8[6], b8[7])) * sc;
     }
-    // Lazy rescale: keep the reference max unless the tile max exceeds it by
-    // more than 8 (log2 units), which bounds P by 2^8.
-    float alpha = 1.f;
-    bool rescale = false;
-    if (mx > m_run + 8.f) {
-      alpha = ex2(m_run - mx);  // 0 when m_run = -inf
-      rescale = (j > 0) && (m_run != -INFINITY);
-      m_run = mx;
-    }
-    const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+    // Weights p = 2^(s * sc - m_ref) against a reference m_ref that is only
+    // raised when the row max exceeds it by more than 8 (log2 units), which
+    // bounds p by 2^8 (lazy rescaling). After the first tile of the unit the
+    // exponentials use the current reference without waiting for this tile's
+    // max; the rare row whose max overshoots is redone with the new one.
     uint32_t pk[32];
     float lt;
-    {
+    auto weights = [&](float m_use) {
       float t[32];
-      if (masked_tile) {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float p0 = ex2(fmaf(s[2 * c], sc, -m_use));
-          const float p1 = ex2(fmaf(s[2 * c + 1], sc, -m_use));
-          pk[c] = POD_PACK(p0, p1);
-          t[c] = p0 + p1;  // unrounded weights (see the decode path)
-        }
-      } else {
-        // kSoftPairs of every 8 column pairs on the FMA pipe, the rest on MUFU
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float x0 = fmaf(s[2 * c], sc, -m_use), x1 = fmaf(s[2 * c + 1], sc, -m_use);
-          const bool soft = (c & 7) >= 8 - kSoftPairs;
-          const float p0 = soft ? exp2_poly(x0) : ex2(x0);
-          const float p1 = soft ? exp2_poly(x1) : ex2(x1);
-          pk[c] = POD_PACK(p0, p1);
-          t[c] = p0 + p1;
-        }
+      for (int c = 0; c < 32; ++c) {
+        const float x0 = fmaf(s[2 * c], sc, -m_use), x1 = fmaf(s[2 * c + 1], sc, -m_use);
+        // kSoftPairs of every 8 column pairs on the FMA pipe (unmasked tiles)
+        const bool soft = !masked_tile && ((c & 7) >= 8 - kSoftPairs);
+        const float p0 = soft ? exp2_poly(x0) : ex2(x0);
+        const float p1 = soft ? exp2_poly(x1) : ex2(x1);
+        pk[c] = POD_PACK(p0, p1);
+        t[c] = p0 + p1;  // unrounded weights (see the decode path)
       }
 #pragma unroll
       for (int w = 16; w >= 1; w >>= 1)
 #pragma unroll
         for (int c = 0; c < w; ++c) t[c] += t[c + w];
       lt = t[0];
+    };
+    float alpha = 1.f;
+    bool rescale = false;
+    if (j == 0 && mx > m_run + 8.f) {  // first tile: the reference comes from it
+      alpha = ex2(m_run - mx);         // 0 when m_run = -inf
+      m_run = mx;
+    }
+    weights((m_run == -INFINITY) ? 0.f : m_run);
+    if (j > 0 && mx > m_run + 8.f) {  // rare: redo this row with a raised reference
+      alpha = ex2(m_run - mx);
+      rescale = (m_run != -INFINITY);
+      m_run = mx;
+      weights(m_run);
     }
     l_run = l_run * alpha + lt;
-    // PV of the previous tile must be done before O is touched and before
-    // the P buffer is overwritten.
+    // PV of the previous tile must be done before O is touched (and waiting
+    // on every completion keeps this thread at most one phase behind).
     if (j > 0) {
       if (!wait_bar_warp(bars + L::B_PV * 8, ps.pv & 1, P, abort_flag)) {
         failed = true;
@@ -752,14 +747,9 @@ POD_DEV bool prefill_softmax(const Plan& P, const PrefillRange& pr, uint8_t* sm,
         tmem_st32(tmem + lane_base + cb * 32, ov);
       }
     }
-    // P (bf16, 128 rows x 64 keys, K-major, 128-byte swizzle) into smem.
-    uint8_t* prow = sm + L::P_OFF + row * 128;
-#pragma unroll
-    for (int ch = 0; ch < 8; ++ch) {
-      uint4 v = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-      *reinterpret_cast<uint4*>(prow + ((ch ^ (row & 7)) << 4)) = v;
-    }
-    fence_proxy_async_smem();
+    // P (bf16 pairs) over the first 32 columns of this tile's S buffer, which
+    // the PV MMA reads as its A operand.
+    tmem_st32(tmem + lane_base + 128 + 64 * b, pk);
     tc_fence_before();
     mbar_arrive(bars + L::B_PF * 8);
   }
@@ -869,7 +859,7 @@ __global__ void __launch_bounds__(kFusedThreads, kFusedSlotsPerSm)
   if (tid == 0) {
     for (int i = 0; i < L::N_BARS; ++i) {
       uint32_t cnt = 1;
-      if (i == L::B_SE || i == L::B_SE + 1 || i == L::B_PF) cnt = 128;
+      if (i == L::B_PF) cnt = 128;  // S-empty barriers: one PV commit each
       mbar_init(bars + i * 8, cnt);
     }
     fence_mbar_init();
