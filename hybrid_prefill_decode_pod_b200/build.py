@@ -16,7 +16,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libpod_attn.so")
 SOURCES = [os.path.join(CSRC, "pod_kernels.cu"), os.path.join(CSRC, "pod_attn_api.cpp"),
            os.path.join(CSRC, "pod_static.cu")]
-HEADERS = [os.path.join(CSRC, f) for f in ("pod_plan.h", "pod_ptx.cuh", "pod_exp2.cuh")] + [
+HEADERS = [os.path.join(CSRC, f) for f in ("pod_plan.h", "pod_ptx.cuh", "pod_exp2.cuh", "pod_prefill.cuh")] + [
     os.path.join(INCLUDE, "pod_attn.h")]
 
 NVCC_FLAGS = [

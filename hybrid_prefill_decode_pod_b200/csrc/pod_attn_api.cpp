@@ -218,13 +218,42 @@ int build_plan(pod_attn_ctx* c, const pod_prefill_args* pa, const pod_decode_arg
   // ---- prefill
   PrefillReq* preq = reinterpret_cast<PrefillReq*>(h + L.preq);
   PrefillUnit* punits = reinterpret_cast<PrefillUnit*>(h + L.punits);
-  long long tiles = 0;
-  for (int p = 0; p < np; ++p) tiles += (long long)((pa->chunk_lens[p] + kQTile - 1) / kQTile) * H;
+  // A unit is two query tiles sharing K/V: a head pair of one KV group at one
+  // token tile (G even) or two consecutive token tiles of one head (G odd).
+  const bool pair_heads = (c->G % 2) == 0;
+  auto tiles_of = [&](int chunk) -> long long {  // pair units of a chunk, one split each
+    const long long qt = (chunk + kQTile - 1) / kQTile;
+    return pair_heads ? qt * (H / 2) : ((qt + 1) / 2) * H;
+  };
+  long long tiles = 0, w_max = 0;
+  for (int p = 0; p < np; ++p) {
+    if (pa->chunk_lens[p] == 0) continue;
+    tiles += tiles_of(pa->chunk_lens[p]);
+    w_max = std::max<long long>(w_max, (pa->prior_lens[p] + pa->chunk_lens[p] + kKVTile - 1) / kKVTile);
+  }
+  // Splits of the KV range (the same count for every request, clamped per
+  // request below): the s minimising the quantised makespan
+  // ceil(U s / slots) (W / s + o) of U units whose longest has W KV tiles, o
+  // being about two tiles of per-unit overhead (Q load, pipeline fill,
+  // epilogue, merge). Only s with U s <= 2 slots are considered, which also
+  // bounds the partial buffers.
   int split_base = 1;
-  if (tiles > 0 && tiles < 2LL * slots) split_base = (int)std::max(1LL, (2LL * slots) / tiles);
+  if (tiles > 0) {
+    double best = 0.0;
+    for (int sp = 1; sp <= kMaxPrefillSplit && tiles * sp <= 2LL * slots; ++sp) {
+      const double waves = (double)((tiles * sp + slots - 1) / slots);
+      const double cost = waves * ((double)w_max / sp + 2.0);
+      if (sp == 1 || cost < 0.97 * best) {
+        best = cost;
+        split_base = sp;
+      }
+    }
+  }
   int n_pu = 0, n_pg = 0, n_ps = 0, max_split = 1, q_row = 0;
   c->units_tmp.clear();
   c->units_key.clear();
+  const int qt_step = pair_heads ? 1 : 2;  // token tiles per unit
+  const int h_step = pair_heads ? 2 : 1;   // heads per unit
   for (int p = 0; p < np; ++p) {
     PrefillReq& R = preq[p];
     const int chunk = pa->chunk_lens[p], prior = pa->prior_lens[p];
@@ -234,15 +263,16 @@ int build_plan(pod_attn_ctx* c, const pod_prefill_args* pa, const pod_decode_arg
     R.n_qtiles = (chunk + kQTile - 1) / kQTile;
     R.kv_len = prior + chunk;
     R.bt_row = p;
+    R.pair_heads = pair_heads ? 1 : 0;
     q_row += chunk;
     if (chunk == 0) {
       R.n_split = 1;
       continue;
     }
-    // smallest tile's KV range, in 64-key tiles; a split keeps >= 16 tiles so
-    // its fixed costs (Q load, pipeline fill, partial write, merge) stay small
-    const int min_tiles = (prior + std::min(chunk, kQTile) + kKVTile - 1) / kKVTile;
-    int split = std::min(split_base, std::max(1, min_tiles / 16));
+    // KV tiles of the request's first unit (its shortest range); a split keeps
+    // >= 4 tiles of 128 keys
+    const int min_tiles = (prior + std::min(chunk, qt_step * kQTile) + kKVTile - 1) / kKVTile;
+    int split = std::min(split_base, std::max(1, min_tiles / 4));
     split = std::min(split, kMaxPrefillSplit);
     R.n_split = split;
     R.n_kvtiles_max = (prior + chunk + kKVTile - 1) / kKVTile;
@@ -253,10 +283,11 @@ int build_plan(pod_attn_ctx* c, const pod_prefill_args* pa, const pod_decode_arg
       n_ps += R.n_qtiles * H * split;
     }
     max_split = std::max(max_split, split);
-    for (int qt = 0; qt < R.n_qtiles; ++qt) {
-      const int kv_hi = prior + std::min(chunk, (qt + 1) * kQTile);
+    for (int qt = 0; qt < R.n_qtiles; qt += qt_step) {
+      const int last_qt = std::min(qt + qt_step, R.n_qtiles) - 1;
+      const int kv_hi = prior + std::min(chunk, (last_qt + 1) * kQTile);
       const int work = (kv_hi + kKVTile - 1) / kKVTile / split;
-      for (int hh = 0; hh < H; ++hh)
+      for (int hh = 0; hh < H; hh += h_step)
         for (int sp = 0; sp < split; ++sp) {
           c->units_tmp.push_back(PrefillUnit{p, hh, qt, sp});
           c->units_key.push_back(work);
@@ -547,7 +578,7 @@ int pod_attn_create(pod_attn_ctx** out, const pod_attn_config* cfg) {
   const long long qtiles = (long long)cfg->max_prefill_tokens / kQTile + cfg->max_prefill_reqs;
   c->cap_punits = (int)std::min<long long>(qtiles * H * kMaxPrefillSplit, 1 << 24);
   c->cap_pgroups = (int)std::min<long long>(std::min<long long>(qtiles * H, 2LL * slots), 1 << 24);
-  c->cap_pslots = 2 * slots + kMaxPrefillSplit * H;  // split only when tiles < 2 waves
+  c->cap_pslots = 4 * slots;  // units x splits <= 2 slots, two query tiles per unit
   c->cap_pgroups = std::max(c->cap_pgroups, 1);
   c->cap_dreqs = std::max(cfg->max_decode_reqs, 1);
   c->cap_dunits = (int)std::max<long long>(16LL * c->num_sms * 8, (long long)c->cap_dreqs * Hk * 2);

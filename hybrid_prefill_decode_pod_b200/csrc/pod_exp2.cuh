@@ -69,4 +69,39 @@ POD_HD float exp2_poly(float x) {
   return i2f_bits((int32_t)((uint32_t)f2i_bits(p) + (uint32_t)f2i_bits(t) * 8388608u));
 }
 
+#ifdef __CUDACC__
+// exp2_poly on both halves of a packed pair with f32x2 instructions. Every
+// step is the scalar version's operation, rounded the same way, so each half
+// equals exp2_poly of that half (f = x - n by one fused multiply-add, exact
+// like the scalar subtraction since |f| <= 0.5).
+__device__ __forceinline__ uint64_t exp2_poly2(float x0, float x1) {
+  x0 = fmaxf(x0, -125.0f);
+  x1 = fmaxf(x1, -125.0f);
+  const float shifter = 12582912.0f;  // 1.5 * 2^23
+  uint64_t x, t, n, f, p, c;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(x0), "f"(x1));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(c) : "f"(shifter));
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(t) : "l"(x), "l"(c));  // t = x + shifter
+  asm("mov.b64 %0, {%1, %1};" : "=l"(c) : "f"(-shifter));
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(n) : "l"(t), "l"(c));  // n = round(x)
+  asm("mov.b64 %0, {%1, %1};" : "=l"(c) : "f"(-1.0f));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(f) : "l"(n), "l"(c), "l"(x));  // f = x - n
+  uint64_t c3, c2;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(c3) : "f"(kExp2C3));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(c2) : "f"(kExp2C2));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(c3), "l"(f), "l"(c2));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(c) : "f"(kExp2C1));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(p), "l"(f), "l"(c));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(c) : "f"(kExp2C0));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(p), "l"(f), "l"(c));
+  uint32_t p0, p1, t0, t1;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(p0), "=r"(p1) : "l"(p));
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(t0), "=r"(t1) : "l"(t));
+  const uint32_t r0 = p0 + t0 * 8388608u, r1 = p1 + t1 * 8388608u;
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(r0), "r"(r1));
+  return r;
+}
+#endif
+
 }  // namespace pod

@@ -88,36 +88,38 @@ POD_DEV void drain_bar(uint32_t bar, uint32_t parity, long long budget) {
 // ============================================================= smem layout
 template <int D>
 struct FusedLayout {
-  static constexpr int QB = kQTile * D * 2;   // Q tile bytes
-  static constexpr int KT = kKVTile * D * 2;  // one K (or V) tile
-  static constexpr int Q_OFF = 0;
-  static constexpr int K_OFF = Q_OFF + QB;                      // K ring
+  static constexpr int QB = kQTile * D * 2;   // one Q tile
+  static constexpr int KT = kKVTile * D * 2;  // one K (or V) tile of 128 keys
+  static constexpr int Q_OFF = 0;                               // Q0, Q1
+  static constexpr int K_OFF = Q_OFF + 2 * QB;                  // K ring
   static constexpr int V_OFF = K_OFF + kPrefillStages * KT;     // V ring
   static constexpr int PREFILL_END = V_OFF + kPrefillStages * KT;
   static constexpr int DEC_ROW = D * 2 + 16;  // padded row: conflict-free ldmatrix
   static constexpr int DEC_STAGE = 2 * kDecTile * DEC_ROW;
   static constexpr int DEC_WARP = kFusedDecStages * DEC_STAGE;
-  static constexpr int DEC_END = kFusedWarps * DEC_WARP;
+  static constexpr int DEC_END = kFusedDecWarps * DEC_WARP;
   static constexpr int DATA_END = PREFILL_END > DEC_END ? PREFILL_END : DEC_END;
   static constexpr int BAR_OFF = (DATA_END + 127) & ~127;
   // barrier indices
-  static constexpr int B_Q = 0;
+  static constexpr int B_Q = 0;                         // Q0 and Q1 landed
   static constexpr int B_KF = 1;                        // K tile landed
-  static constexpr int B_KE = B_KF + kPrefillStages;    // K tile consumed by S = Q K^T
+  static constexpr int B_KE = B_KF + kPrefillStages;    // K tile read by both S MMAs
   static constexpr int B_VF = B_KE + kPrefillStages;    // V tile landed
-  static constexpr int B_VE = B_VF + kPrefillStages;    // V tile consumed by O += P V
-  static constexpr int B_SF = B_VE + kPrefillStages;
-  static constexpr int B_SE = B_SF + 2;                 // S buffer free (its P consumed by PV)
-  static constexpr int B_PF = B_SE + 2;
-  static constexpr int B_PV = B_PF + 1;
-  static constexpr int B_DEC = B_PV + 1;
-  static constexpr int N_BARS = B_DEC + kFusedWarps * kFusedDecStages;
+  static constexpr int B_VE = B_VF + kPrefillStages;    // V tile read by both PV MMAs
+  static constexpr int B_SF = B_VE + kPrefillStages;    // S_i in TMEM [2]
+  static constexpr int B_SE = B_SF + 2;                 // S_i free (its P read by PV_i) [2]
+  static constexpr int B_PF = B_SE + 2;                 // P_i in TMEM, one arrival per warp [2]
+  static constexpr int B_OR = B_PF + 2;                 // O_i final for the unit [2]
+  static constexpr int B_DEC = B_OR + 2;
+  static constexpr int N_BARS = B_DEC + kFusedDecWarps * kFusedDecStages;
   static constexpr int MISC_OFF = BAR_OFF + N_BARS * 8;
   static constexpr int TOTAL = MISC_OFF + 64;
+  static_assert(TOTAL <= 227 * 1024, "fused CTA exceeds the shared memory of an SM");
   // The dynamic shared memory window of a CTA without static shared memory
   // starts 1024-byte aligned; the kernel checks it and refuses to run (status)
-  // otherwise. No slack is added: two CTAs must fit in one SM.
-  static constexpr int SMEM_BYTES = TOTAL;
+  // otherwise. At least 116 KB are requested so that two CTAs never share an
+  // SM (2 x 117 KB > 228 KB): each CTA holds all 512 TMEM columns for its life.
+  static constexpr int SMEM_BYTES = TOTAL > 116 * 1024 ? TOTAL : 116 * 1024;
 };
 
 template <int D>
@@ -462,377 +464,7 @@ POD_DEV bool decode_unit_warp(const Plan& P, int u, uint8_t* wsm, uint32_t bar0,
 }
 
 // ============================================================= prefill unit
-struct PrefillRange {
-  int req, head, qtile, split;
-  int t0, n;  // first KV tile and number of KV tiles
-};
-
-POD_DEV PrefillRange prefill_range(const Plan& P, int u) {
-  const PrefillUnit U = P.punits[u];
-  const PrefillReq R = P.preq[U.req];
-  const int kv_hi = R.prior + min(R.chunk, (U.qtile + 1) * kQTile);
-  const int n_all = (kv_hi + kKVTile - 1) / kKVTile;
-  PrefillRange pr;
-  pr.req = U.req;
-  pr.head = U.head;
-  pr.qtile = U.qtile;
-  pr.split = U.split;
-  pr.t0 = (int)((long long)U.split * n_all / R.n_split);
-  pr.n = (int)((long long)(U.split + 1) * n_all / R.n_split) - pr.t0;
-  return pr;
-}
-
-// Per-CTA iteration counters that carry mbarrier phases across units.
-struct PipeState {
-  uint32_t kv;       // KV tiles processed
-  uint32_t q;        // Q tiles loaded
-  uint32_t pv;       // PV completions observed by softmax threads
-  uint32_t kissued;  // producer: K tiles issued (for the abort drain)
-  uint32_t vissued;  // producer: V tiles issued
-};
-
-// ---- TMA producer (one thread). Two rings: a K stage is released as soon as
-// S = Q K^T has read it, a V stage once O += P V has; K runs one tile ahead.
-template <int D>
-POD_DEV bool prefill_producer(const Plan& P, const TmaDescs& T, const PrefillRange& pr,
-                              uint8_t* sm, PipeState& ps, volatile int* abort_flag) {
-  using L = FusedLayout<D>;
-  const uint32_t base = smem_u32(sm);
-  const uint32_t bars = base + L::BAR_OFF;
-  const PrefillReq R = P.preq[pr.req];
-  const int g = pr.head / P.G;
-  constexpr int NB = D / 64;  // 64-column swizzle blocks
-  // Q tile
-  mbar_expect_tx(bars + L::B_Q * 8, L::QB);
-  for (int b = 0; b < NB; ++b)
-    tma_load_3d(base + L::Q_OFF + b * (kQTile * 128), &T.q, bars + L::B_Q * 8, 64 * b, pr.head,
-                R.q_row0 + pr.qtile * kQTile);
-  ps.q++;
-  const CUtensorMap* km = P.paged ? &T.k[0] : &T.k[pr.req];
-  const CUtensorMap* vm = P.paged ? &T.v[0] : &T.v[pr.req];
-  const int last_page = (R.kv_len - 1) >> 4;
-
-  // one K or V tile of 64 keys into ring `off` stage `st`, completing on `full`
-  auto load_tile = [&](const CUtensorMap* m, uint32_t dst, uint32_t full, int key0) {
-    mbar_expect_tx(full, L::KT);
-    if (!P.paged) {
-      for (int b = 0; b < NB; ++b) tma_load_3d(dst + b * (kKVTile * 128), m, full, 64 * b, g, key0);
-    } else {
-      for (int pg = 0; pg < kKVTile / 16; ++pg) {
-        const int lp = min((key0 >> 4) + pg, last_page);
-        const int phys = __ldg(P.bt_p + (size_t)R.bt_row * P.bt_stride_p + lp);
-        for (int b = 0; b < NB; ++b)
-          tma_load_3d(dst + b * (kKVTile * 128) + pg * 16 * 128, m, full, 64 * b, g, phys * 16);
-      }
-    }
-  };
-  auto issue = [&](int j, bool is_k) -> bool {
-    const uint32_t it = ps.kv + j;
-    const uint32_t st = it % kPrefillStages;
-    const uint32_t ph = (it / kPrefillStages) & 1;
-    const int empty = is_k ? L::B_KE : L::B_VE;
-    if (it >= kPrefillStages && !wait_bar(bars + (empty + st) * 8, ph ^ 1, P, abort_flag))
-      return false;
-    const uint32_t dst = base + (is_k ? L::K_OFF : L::V_OFF) + st * L::KT;
-    load_tile(is_k ? km : vm, dst, bars + ((is_k ? L::B_KF : L::B_VF) + st) * 8,
-              (pr.t0 + j) * kKVTile);
-    return true;
-  };
-  bool ok = issue(0, true);
-  ps.kissued = ps.kv + 1;
-  for (int j = 0; ok && j < pr.n; ++j) {
-    if (j + 1 < pr.n) {
-      ok = issue(j + 1, true);
-      if (ok) ps.kissued = ps.kv + j + 2;
-    }
-    if (ok) {
-      ok = issue(j, false);
-      if (ok) ps.vissued = ps.kv + j + 1;
-    }
-  }
-  ps.kv += pr.n;
-  return ok;
-}
-
-template <int D>
-POD_DEV void prefill_producer_drain(const Plan& P, uint8_t* sm, const PipeState& ps) {
-  using L = FusedLayout<D>;
-  const uint32_t bars = smem_u32(sm) + L::BAR_OFF;
-  if (ps.q > 0) drain_bar(bars + L::B_Q * 8, (ps.q - 1) & 1, P.wait_budget);
-  for (uint32_t k = 0; k < kPrefillStages && k < ps.kissued; ++k) {
-    const uint32_t it = ps.kissued - 1 - k;
-    drain_bar(bars + (L::B_KF + it % kPrefillStages) * 8, (it / kPrefillStages) & 1,
-              P.wait_budget);
-  }
-  for (uint32_t k = 0; k < kPrefillStages && k < ps.vissued; ++k) {
-    const uint32_t it = ps.vissued - 1 - k;
-    drain_bar(bars + (L::B_VF + it % kPrefillStages) * 8, (it / kPrefillStages) & 1,
-              P.wait_budget);
-  }
-}
-
-// ---- MMA issuer (one thread)
-template <int D>
-POD_DEV bool prefill_mma(const Plan& P, const PrefillRange& pr, uint8_t* sm, uint32_t tmem,
-                         PipeState& ps, uint32_t& last_commit_bar, uint32_t& last_commit_par,
-                         volatile int* abort_flag) {
-  using L = FusedLayout<D>;
-  constexpr int KS = D / 16;
-  constexpr uint32_t IDESC_QK = umma_idesc_bf16(kQTile, kKVTile, 0, 0);
-  constexpr uint32_t IDESC_PV = umma_idesc_bf16(kQTile, D, 0, 1);
-  const uint32_t base = smem_u32(sm);
-  const uint32_t bars = base + L::BAR_OFF;
-  if (!wait_bar(bars + L::B_Q * 8, ps.q & 1, P, abort_flag)) return false;
-  ps.q++;
-  tc_fence_after();
-
-  auto issue_pv = [&](int jj) -> bool {
-    const uint32_t it = ps.kv + jj;
-    const uint32_t st = it % kPrefillStages, ph = (it / kPrefillStages) & 1;
-    if (!wait_bar(bars + L::B_PF * 8, it & 1, P, abort_flag)) return false;
-    if (!wait_bar(bars + (L::B_VF + st) * 8, ph, P, abort_flag)) return false;
-    tc_fence_after();
-    const uint32_t vbase = base + L::V_OFF + st * L::KT;
-    // P (bf16 pairs) sits in the first 32 columns of the S buffer it came from
-    const uint32_t pcol = tmem + 128 + 64 * (it & 1);
-#pragma unroll
-    for (int kk = 0; kk < kKVTile / 16; ++kk) {
-      const uint64_t bd = sw128_desc(vbase + kk * 16 * 128, kKVTile * 128, 1024);
-      umma_ts(tmem + 0, pcol + kk * 8, bd, IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
-    }
-    umma_commit(bars + L::B_PV * 8);
-    umma_commit(bars + (L::B_VE + st) * 8);
-    umma_commit(bars + (L::B_SE + (it & 1)) * 8);  // S buffer free once its P is consumed
-    last_commit_bar = bars + L::B_PV * 8;
-    last_commit_par = it & 1;  // pv_done completes once per tile
-    return true;
-  };
-
-  for (int j = 0; j < pr.n; ++j) {
-    const uint32_t it = ps.kv + j;
-    const uint32_t st = it % kPrefillStages, ph = (it / kPrefillStages) & 1;
-    const uint32_t b = it & 1;
-    if (!wait_bar(bars + (L::B_KF + st) * 8, ph, P, abort_flag)) return false;
-    if (it >= 2 && !wait_bar(bars + (L::B_SE + b) * 8, ((it >> 1) - 1) & 1, P, abort_flag))
-      return false;
-    tc_fence_after();
-    const uint32_t kbase = base + L::K_OFF + st * L::KT;
-#pragma unroll
-    for (int kk = 0; kk < KS; ++kk) {
-      const uint64_t ad = sw128_desc(base + L::Q_OFF + (kk >> 2) * (kQTile * 128) + (kk & 3) * 32,
-                                     16, 1024);
-      const uint64_t bd = sw128_desc(kbase + (kk >> 2) * (kKVTile * 128) + (kk & 3) * 32, 16, 1024);
-      umma_ss(tmem + 128 + 64 * b, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
-    }
-    umma_commit(bars + (L::B_SF + b) * 8);
-    umma_commit(bars + (L::B_KE + st) * 8);  // K stage free once S has read it
-    last_commit_bar = bars + (L::B_SF + b) * 8;
-    last_commit_par = (it >> 1) & 1;
-    if (j > 0 && !issue_pv(j - 1)) return false;
-  }
-  if (!issue_pv(pr.n - 1)) return false;
-  ps.kv += pr.n;
-  return true;
-}
-
-// ---- softmax + epilogue (128 threads, thread = query row = TMEM lane)
-template <int D>
-POD_DEV bool prefill_softmax(const Plan& P, const PrefillRange& pr, uint8_t* sm, uint32_t tmem,
-                             PipeState& ps, int tid, volatile int* abort_flag, int* s_flag) {
-  using L = FusedLayout<D>;
-  const uint32_t base = smem_u32(sm);
-  const uint32_t bars = base + L::BAR_OFF;
-  const PrefillReq R = P.preq[pr.req];
-  const int warp = tid >> 5;
-  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-  const int row = tid;
-  const int q_local = pr.qtile * kQTile + row;  // token index within the chunk
-  const int lim = R.prior + q_local;            // last visible key (inclusive)
-  const int mask_from = R.prior + pr.qtile * kQTile;  // tiles ending above this need masking
-  const float sc = P.scale_log2;
-  float m_run = -INFINITY, l_run = 0.f;
-  bool failed = false;  // warp-uniform; after a failure only barrier points are kept
-
-  for (int j = 0; j < pr.n; ++j) {
-    const uint32_t it = ps.kv + j;
-    const uint32_t b = it & 1;
-    if (!wait_bar_warp(bars + (L::B_SF + b) * 8, (it >> 1) & 1, P, abort_flag)) {
-      failed = true;
-      break;
-    }
-    tc_fence_after();
-    uint32_t sr[2][32];
-    tmem_ld32x2(tmem + lane_base + 128 + 64 * b, sr[0], sr[1]);
-
-    const int key0 = (pr.t0 + j) * kKVTile;
-    float s[64];
-#pragma unroll
-    for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(sr[c >> 5][c & 31]);
-    const bool masked_tile = key0 + kKVTile - 1 > mask_from;  // uniform over the CTA
-    if (masked_tile) {
-#pragma unroll
-      for (int c = 0; c < 64; ++c)
-        if (key0 + c > lim) s[c] = -INFINITY;
-    }
-    float mx;
-    {  // 64 -> 22 -> 8 -> 3 -> 1 with three-input max
-      float a[22], b8[8];
-#pragma unroll
-      for (int c = 0; c < 21; ++c) a[c] = max3(s[3 * c], s[3 * c + 1], s[3 * c + 2]);
-      a[21] = s[63];
-#pragma unroll
-      for (int c = 0; c < 7; ++c) b8[c] = max3(a[3 * c], a[3 * c + 1], a[3 * c + 2]);
-      b8[7] = a[21];
-      mx = max3(max3(b8[0], b8[1], b8[2]), max3(b8[3], b8[4], b8[5]), fmaxf(b8[6], b8[7])) * sc;
-    }
-    // Weights p = 2^(s * sc - m_ref) against a reference m_ref that is only
-    // raised when the row max exceeds it by more than 8 (log2 units), which
-    // bounds p by 2^8 (lazy rescaling). After the first tile of the unit the
-    // exponentials use the current reference without waiting for this tile's
-    // max; the rare row whose max overshoots is redone with the new one.
-    uint32_t pk[32];
-    float lt;
-    auto weights = [&](float m_use) {
-      float t[32];
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const float x0 = fmaf(s[2 * c], sc, -m_use), x1 = fmaf(s[2 * c + 1], sc, -m_use);
-        // kSoftPairs of every 8 column pairs on the FMA pipe (unmasked tiles)
-        const bool soft = !masked_tile && ((c & 7) >= 8 - kSoftPairs);
-        const float p0 = soft ? exp2_poly(x0) : ex2(x0);
-        const float p1 = soft ? exp2_poly(x1) : ex2(x1);
-        pk[c] = POD_PACK(p0, p1);
-        t[c] = p0 + p1;  // unrounded weights (see the decode path)
-      }
-#pragma unroll
-      for (int w = 16; w >= 1; w >>= 1)
-#pragma unroll
-        for (int c = 0; c < w; ++c) t[c] += t[c + w];
-      lt = t[0];
-    };
-    float alpha = 1.f;
-    bool rescale = false;
-    if (j == 0 && mx > m_run + 8.f) {  // first tile: the reference comes from it
-      alpha = ex2(m_run - mx);         // 0 when m_run = -inf
-      m_run = mx;
-    }
-    weights((m_run == -INFINITY) ? 0.f : m_run);
-    if (j > 0 && mx > m_run + 8.f) {  // rare: redo this row with a raised reference
-      alpha = ex2(m_run - mx);
-      rescale = (m_run != -INFINITY);
-      m_run = mx;
-      weights(m_run);
-    }
-    l_run = l_run * alpha + lt;
-    // PV of the previous tile must be done before O is touched (and waiting
-    // on every completion keeps this thread at most one phase behind).
-    if (j > 0) {
-      if (!wait_bar_warp(bars + L::B_PV * 8, ps.pv & 1, P, abort_flag)) {
-        failed = true;
-        break;
-      }
-      ps.pv++;
-      tc_fence_after();
-    }
-    // tcgen05.ld/st are warp-collective (.sync.aligned): the whole warp takes
-    // this branch if any of its rows must rescale; the others multiply by 1.
-    if (__any_sync(0xffffffffu, rescale)) {
-      const float f = rescale ? alpha : 1.f;
-#pragma unroll
-      for (int cb = 0; cb < D / 32; ++cb) {
-        uint32_t ov[32];
-        tmem_ld32(tmem + lane_base + cb * 32, ov);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * f);
-        tmem_st32(tmem + lane_base + cb * 32, ov);
-      }
-    }
-    // P (bf16 pairs) over the first 32 columns of this tile's S buffer, which
-    // the PV MMA reads as its A operand.
-    tmem_st32(tmem + lane_base + 128 + 64 * b, pk);
-    tc_fence_before();
-    mbar_arrive(bars + L::B_PF * 8);
-  }
-  // final PV
-  if (!failed) {
-    if (wait_bar_warp(bars + L::B_PV * 8, ps.pv & 1, P, abort_flag)) {
-      ps.pv++;
-      tc_fence_after();
-    } else {
-      failed = true;
-    }
-  }
-  ps.kv += pr.n;
-
-  const PrefillReq& RR = R;
-  const bool valid = (q_local < RR.chunk) && !failed;
-  const size_t out_row = (size_t)(RR.q_row0 + q_local);
-  const float lse2 = (l_run > 0.f) ? (m_run + log2f(l_run)) : -INFINITY;
-  if (RR.n_split <= 1) {
-    if (failed) return false;
-    const float inv = 1.f / l_run;
-#pragma unroll
-    for (int cb = 0; cb < D / 32; ++cb) {
-      uint32_t ov[32];
-      tmem_ld32(tmem + lane_base + cb * 32, ov);
-      if (valid) {
-        uint16_t* dst = P.o_p + (out_row * P.H + pr.head) * D + cb * 32;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint4 v;
-          v.x = pack_bf16(__uint_as_float(ov[8 * q + 0]) * inv, __uint_as_float(ov[8 * q + 1]) * inv);
-          v.y = pack_bf16(__uint_as_float(ov[8 * q + 2]) * inv, __uint_as_float(ov[8 * q + 3]) * inv);
-          v.z = pack_bf16(__uint_as_float(ov[8 * q + 4]) * inv, __uint_as_float(ov[8 * q + 5]) * inv);
-          v.w = pack_bf16(__uint_as_float(ov[8 * q + 6]) * inv, __uint_as_float(ov[8 * q + 7]) * inv);
-          *reinterpret_cast<uint4*>(dst + 8 * q) = v;
-        }
-      }
-    }
-    if (valid) P.lse_p[out_row * P.H + pr.head] = lse2 * kLn2;
-    return true;
-  }
-  // split partial: normalised O (fp32) and LSE of this KV range
-  const int gidx = pr.qtile * P.H + pr.head;
-  const int slot = RR.slot0 + gidx * RR.n_split + pr.split;
-  const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
-  float* po = P.ppart_o + ((size_t)slot * kQTile + row) * D;
-#pragma unroll
-  for (int cb = 0; cb < D / 32 && !failed; ++cb) {
-    uint32_t ov[32];
-    tmem_ld32(tmem + lane_base + cb * 32, ov);
-    if (valid) {
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        float4 v = make_float4(__uint_as_float(ov[4 * q]) * inv, __uint_as_float(ov[4 * q + 1]) * inv,
-                               __uint_as_float(ov[4 * q + 2]) * inv,
-                               __uint_as_float(ov[4 * q + 3]) * inv);
-        *reinterpret_cast<float4*>(po + cb * 32 + 4 * q) = v;
-      }
-    }
-  }
-  if (valid) P.ppart_lse[(size_t)slot * kQTile + row] = lse2 * kLn2;
-  __threadfence();
-  asm volatile("bar.sync 1, 128;" ::: "memory");
-  if (tid == 0) {
-    // after a failure nobody merges (the group can never be complete)
-    const int old = *abort_flag ? -1 : atomicAdd(P.pgroup_ctr + RR.group0 + gidx, 1);
-    *s_flag = (old == RR.n_split - 1);
-  }
-  asm volatile("bar.sync 1, 128;" ::: "memory");
-  if (*s_flag && !failed) {
-    __threadfence();
-    const int rows = min(kQTile, RR.chunk - pr.qtile * kQTile);
-    const int slot0 = RR.slot0 + gidx * RR.n_split;
-    const size_t orow0 = (size_t)(RR.q_row0 + pr.qtile * kQTile);
-    // warp w merges rows [32w, 32w + 32), four at a time
-    for (int i0 = warp * 32; i0 < min(rows, warp * 32 + 32); i0 += 4)
-      merge_rows_warp<D, 4>(P.ppart_o + (size_t)slot0 * kQTile * D, (long long)kQTile * D, D,
-                            P.ppart_lse + (size_t)slot0 * kQTile, kQTile, 1, RR.n_split, i0,
-                            min(rows, warp * 32 + 32), P.o_p + (orow0 * P.H + pr.head) * D,
-                            (long long)P.H * D, P.lse_p + orow0 * P.H + pr.head, P.H, tid & 31);
-  }
-  return !failed;
-}
+#include "pod_prefill.cuh"
 
 // ============================================================= fused kernel
 // Roles: PREFILL = 1, DECODE = 2. allow_prefill / allow_decode restrict the
@@ -852,14 +484,14 @@ __global__ void __launch_bounds__(kFusedThreads, kFusedSlotsPerSm)
   const int warp = tid >> 5, lane = tid & 31;
   const uint32_t bars = smem_u32(sm) + L::BAR_OFF;
   int* misc = reinterpret_cast<int*>(sm + L::MISC_OFF);
-  // misc[0] tmem addr, [1] role, [2] unit, [3] abort flag, [4] merge flag,
-  // [5] prefill queue empty, [6] decode queue empty
+  // misc[0] tmem addr, [1] role, [2] unit, [3] abort flag, [5] prefill queue
+  // empty, [6] decode queue empty, [7..8] merge flags of the two query tiles
   volatile int* abort_flag = misc + 3;
 
   if (tid == 0) {
     for (int i = 0; i < L::N_BARS; ++i) {
       uint32_t cnt = 1;
-      if (i == L::B_PF) cnt = 128;  // S-empty barriers: one PV commit each
+      if (i == L::B_PF || i == L::B_PF + 1) cnt = kSoftmaxWarps / 2;  // one per softmax warp
       mbar_init(bars + i * 8, cnt);
     }
     fence_mbar_init();
@@ -902,7 +534,7 @@ __global__ void __launch_bounds__(kFusedThreads, kFusedSlotsPerSm)
         const int t = atomicAdd(P.sm_ticket + ((P.flags & 0x100) ? 0 : my_sm), 1);
         const long long num = P.rho_num, den = P.rho_den > 0 ? P.rho_den : 1;
         bool want_p = ((long long)(t + 1) * num) / den > ((long long)t * num) / den;
-        // front-loaded: each SM's first two tickets (one per resident CTA) take
+        // front-loaded: each SM's first ticket (one per resident CTA) takes
         // prefill work, so the long prefill units start first
         if ((P.flags & 0x200) && t < kFusedSlotsPerSm) want_p = true;
         for (int attempt = 0; attempt < 2 && role == 0; ++attempt, want_p = !want_p) {
@@ -930,9 +562,9 @@ __global__ void __launch_bounds__(kFusedThreads, kFusedSlotsPerSm)
     if (role == 0) break;
     if (role == 1) {
       const PrefillRange pr = prefill_range(P, unit);
-      if (warp < 4) {
-        prefill_softmax<D>(P, pr, sm, tmem, ps, tid, abort_flag, misc + 4);
-      } else if (warp == 4) {
+      if (warp < kSoftmaxWarps) {
+        prefill_softmax<D>(P, pr, sm, tmem, ps, tid, abort_flag, misc + 7);
+      } else if (warp == kSoftmaxWarps) {
         if (lane == 0) {
           issued_mma = true;
           prefill_mma<D>(P, pr, sm, tmem, ps, last_commit_bar, last_commit_par, abort_flag);
@@ -969,8 +601,8 @@ __global__ void __launch_bounds__(kFusedThreads, kFusedSlotsPerSm)
   }
   // Teardown. After an abort, wait (bounded) for this CTA's own async work.
   if (*abort_flag) {
-    if (warp == 5 && lane == 0) prefill_producer_drain<D>(P, sm, ps);
-    if (warp == 4 && lane == 0 && issued_mma && last_commit_bar)
+    if (warp == kSoftmaxWarps + 1 && lane == 0) prefill_producer_drain<D>(P, sm, ps);
+    if (warp == kSoftmaxWarps && lane == 0 && issued_mma && last_commit_bar)
       drain_bar(last_commit_bar, last_commit_par, P.wait_budget);
   }
   tc_fence_before();

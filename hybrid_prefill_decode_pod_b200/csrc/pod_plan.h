@@ -16,26 +16,33 @@ namespace pod {
 
 constexpr int kMaxPrefillReqs = 16;
 constexpr int kQTile = 128;           // prefill query rows per unit (= UMMA M)
-constexpr int kKVTile = 64;           // prefill keys per KV tile (= UMMA N of S)
+constexpr int kKVTile = 128;          // prefill keys per KV tile (= UMMA N of S)
 constexpr int kPrefillStages = 2;     // K/V smem ring depth in the prefill role
 constexpr int kDecTile = 16;          // decode keys per staged tile (= mma M)
-constexpr int kFusedWarps = 6;        // 4 softmax + 1 MMA issuer + 1 TMA producer
+constexpr int kFusedWarps = 10;       // 8 softmax (2 query tiles) + MMA issuer + TMA producer
 constexpr int kFusedThreads = kFusedWarps * 32;
-constexpr int kFusedSlotsPerSm = 2;   // persistent CTAs per SM
+constexpr int kSoftmaxWarps = 8;
+constexpr int kFusedDecWarps = 10;    // every warp is a virtual decode unit in a decode turn
+constexpr int kFusedSlotsPerSm = 1;   // persistent CTAs per SM (the CTA owns all TMEM)
+static_assert(kFusedWarps == kSoftmaxWarps + 2, "softmax warps + MMA issuer + producer");
+static_assert(kFusedDecWarps == kFusedWarps, "a decode turn runs on every warp");
 constexpr int kFusedDecStages = 2;    // per-warp decode ring depth in the fused kernel
 constexpr int kDecodeWarps = 6;       // warps (virtual decode units) per decode-only CTA
 constexpr int kDecodeStages = 2;      // per-warp ring depth in the decode-only kernel
 constexpr int kMaxGroup = 8;          // query heads per KV head (mma N = 8)
-constexpr int kTmemCols = 256;        // TMEM columns per CTA: O [0,128), S0, S1 [128,256)
+constexpr int kTmemCols = 512;        // TMEM columns per CTA: O0, O1, S0, S1 (128 each)
 constexpr int kMaxSmid = 256;         // per-SM ticket slots (indexed by %smid)
 constexpr long long kDefaultWaitBudget = 2000000000LL;  // cycles (~1 s at 2 GHz)
 
 struct PrefillReq {
   int prior, chunk, q_row0, n_qtiles;
   int kv_len, bt_row, n_split, group0;  // group0: first merge group of this request
-  int slot0, n_kvtiles_max, pad0, pad1; // slot0: first partial slot (split requests)
+  int slot0, n_kvtiles_max, pair_heads, pad1;  // slot0: first partial slot (split
+                                               // requests); pair_heads: see PrefillUnit
 };
 
+// Two query tiles: heads (head, head + 1) at token tile qtile when the
+// request's pair_heads is set, else token tiles (qtile, qtile + 1) of head.
 struct PrefillUnit {
   int req, head, qtile, split;
 };
