@@ -73,6 +73,7 @@ struct pod_attn_ctx {
   // scheduling levers (defaults; environment overrides exist for ablations)
   int policy = 4;        // 0 proportional, 1 even (50:50), 2 prefill first, 3 decode first,
                          // 4 front (each SM's first tickets take prefill, then 50:50)
+                         // 5 balanced (a fixed set of SMs takes prefill first)
   int smid_aware = 1;    // per-SM tickets (1) or one global ticket counter (0)
   int dec_turn = 1;      // decode units each warp claims per decode turn of a fused CTA
   int dec_split = 0;     // 0: cost model; else keys per decode split (multiple of 16)
@@ -380,6 +381,24 @@ int build_plan(pod_attn_ctx* c, const pod_prefill_args* pa, const pod_decode_arg
   if (c->policy == 2) { rho_num = 1; rho_den = 1; }
   if (c->policy == 3) { rho_num = 0; rho_den = 1; }
   if (c->policy == 4) { rho_num = 1; rho_den = 2; }  // front: see pod_fused_kernel
+  // balanced (POD-Attention §4.1: match the prefill and decode shares of the
+  // SMs to their work): CTAs 0..p_cap-1 take prefill first, the others decode
+  // first. With the decode side bound by HBM, decode alone takes about
+  // bytes / bandwidth on the whole GPU and still about that on the SMs left
+  // to it, as long as those are enough to keep HBM busy; prefill needs
+  // sum(unit times) SM-microseconds. p_cap is the SM count on which prefill
+  // finishes in the decode time (all SMs when prefill dominates).
+  int p_cap = slots;
+  if (c->policy == 5 && n_pu > 0 && nd > 0) {
+    const double tile_us = (c->D == 128 ? 2.0 : 1.2), unit_us = 3.0;
+    double p_sm_us = 0.0;
+    for (int u = 0; u < n_pu; ++u) p_sm_us += c->units_key[u] * tile_us + unit_us;
+    double kv_keys = 0.0;
+    for (int r = 0; r < nd; ++r) kv_keys += (double)da->ctx_lens[r];
+    const double d_us = kv_keys * Hk * c->D * 4.0 / 6.0e6;  // K and V, bf16, ~6 TB/s
+    if (d_us > p_sm_us / slots)
+      p_cap = std::max(1, std::min(slots, (int)std::ceil(p_sm_us / d_us)));
+  }
   if (rho_den == 0) rho_den = 1;
 
   // ---- kernel parameters
@@ -400,7 +419,9 @@ int build_plan(pod_attn_ctx* c, const pod_prefill_args* pa, const pod_decode_arg
   Q.paged = paged ? 1 : 0;
   Q.bt_stride_p = (np && paged) ? pa->block_table_stride : 0;
   Q.bt_stride_d = (nd && paged) ? da->block_table_stride : 0;
-  Q.flags = (int)c->cfg.flags | (c->smid_aware ? 0 : 0x100) | (c->policy == 4 ? 0x200 : 0);
+  Q.flags = (int)c->cfg.flags | (c->smid_aware ? 0 : 0x100) | (c->policy == 4 ? 0x200 : 0) |
+            (c->policy == 5 ? 0x400 : 0);
+  Q.p_cap = p_cap;
   Q.dec_turn = c->dec_turn;
   Q.wait_budget = kDefaultWaitBudget;
   char* dp = c->d_plan;
@@ -470,6 +491,7 @@ int build_plan(pod_attn_ctx* c, const pod_prefill_args* pa, const pod_decode_arg
   c->last.decode_split_len = nd ? split_len : 0;
   c->last.ratio_num = rho_num;
   c->last.ratio_den = rho_den;
+  c->last.prefill_sm_cap = p_cap;
   size_t used = L.dunit + sizeof(int) * (size_t)n_du;
   if (n_du == 0) used = L.dreq + sizeof(DecodeReq) * (size_t)nd;
   if (nd == 0 && n_du == 0) used = L.punits + sizeof(PrefillUnit) * (size_t)n_pu;
@@ -563,6 +585,7 @@ int pod_attn_create(pod_attn_ctx** out, const pod_attn_config* cfg) {
     else if (!std::strcmp(e, "prefill_first")) c->policy = 2;
     else if (!std::strcmp(e, "decode_first")) c->policy = 3;
     else if (!std::strcmp(e, "front")) c->policy = 4;
+    else if (!std::strcmp(e, "balanced")) c->policy = 5;
     else if (!std::strcmp(e, "proportional")) c->policy = 0;
   }
   if (const char* e = std::getenv("POD_ATTN_SMID_AWARE")) c->smid_aware = std::atoi(e) != 0;

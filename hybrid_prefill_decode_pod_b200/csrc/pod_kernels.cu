@@ -537,6 +537,9 @@ __global__ void __launch_bounds__(kFusedThreads, kFusedSlotsPerSm)
         // front-loaded: each SM's first ticket (one per resident CTA) takes
         // prefill work, so the long prefill units start first
         if ((P.flags & 0x200) && t < kFusedSlotsPerSm) want_p = true;
+        // balanced: a fixed set of CTAs (one per SM) serves prefill first and
+        // the rest serve decode first, sized so both finish together
+        if (P.flags & 0x400) want_p = (int)blockIdx.x < P.p_cap;
         for (int attempt = 0; attempt < 2 && role == 0; ++attempt, want_p = !want_p) {
           if (want_p && !misc[5]) {
             const int u = atomicAdd(P.ctl + 0, 1);
@@ -570,10 +573,11 @@ __global__ void __launch_bounds__(kFusedThreads, kFusedSlotsPerSm)
           prefill_mma<D>(P, pr, sm, tmem, ps, last_commit_bar, last_commit_par, abort_flag);
         }
         __syncwarp();
-      } else {
+      } else if (warp == kSoftmaxWarps + 1) {
         if (lane == 0) prefill_producer<D>(P, T, pr, sm, ps, abort_flag);
         __syncwarp();
       }
+      // warps past the producer have no prefill role; they run decode turns
     } else {
       // decode turn: every warp is a virtual decode unit runner and claims up
       // to dec_turn units one at a time; once every prefill unit has been

@@ -19,12 +19,13 @@ constexpr int kQTile = 128;           // prefill query rows per unit (= UMMA M)
 constexpr int kKVTile = 128;          // prefill keys per KV tile (= UMMA N of S)
 constexpr int kPrefillStages = 2;     // K/V smem ring depth in the prefill role
 constexpr int kDecTile = 16;          // decode keys per staged tile (= mma M)
-constexpr int kFusedWarps = 10;       // 8 softmax (2 query tiles) + MMA issuer + TMA producer
+constexpr int kFusedWarps = 12;       // 8 softmax (2 query tiles) + MMA issuer + TMA producer + 2
+                                      // more decode runners (3 warps per SM sub-partition either way)
 constexpr int kFusedThreads = kFusedWarps * 32;
 constexpr int kSoftmaxWarps = 8;
-constexpr int kFusedDecWarps = 10;    // every warp is a virtual decode unit in a decode turn
+constexpr int kFusedDecWarps = 12;    // every warp is a virtual decode unit in a decode turn
 constexpr int kFusedSlotsPerSm = 1;   // persistent CTAs per SM (the CTA owns all TMEM)
-static_assert(kFusedWarps == kSoftmaxWarps + 2, "softmax warps + MMA issuer + producer");
+static_assert(kFusedWarps >= kSoftmaxWarps + 2, "softmax warps + MMA issuer + producer");
 static_assert(kFusedDecWarps == kFusedWarps, "a decode turn runs on every warp");
 constexpr int kFusedDecStages = 2;    // per-warp decode ring depth in the fused kernel
 constexpr int kDecodeWarps = 6;       // warps (virtual decode units) per decode-only CTA
@@ -67,7 +68,7 @@ struct Plan {
   int flags;
   int pool_blocks;               // paged: blocks in the pool (bounds every block id)
   int dec_turn;                  // decode units per warp per fused decode turn
-  int pad1;
+  int p_cap;                     // balanced policy: CTAs 0..p_cap-1 take prefill first
   long long wait_budget;         // cycles a bounded wait may spin
   const PrefillReq* preq;
   const PrefillUnit* punits;

@@ -386,26 +386,29 @@ POD_DEV bool prefill_softmax(const Plan& P, const PrefillRange& pr, uint8_t* sm,
     if (valid) P.lse_p[out_row * P.H + head] = lse2 * kLn2;
     return true;
   }
-  // split partial of this tile: normalised O (fp32) and the LSE of its KV range
+  // Split partial of this tile: O normalised by its own sum (fp32) and the
+  // natural-log LSE of its KV range. O is stored [slot][d / 4][row] in float4
+  // units, so the 32 rows of a warp touch 512 contiguous bytes per access.
   const int gidx = qtile * P.H + head;
-  const int slot = R.slot0 + gidx * R.n_split + pr.split;
+  const int slot0 = R.slot0 + gidx * R.n_split;
   const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
-  float* po = P.ppart_o + ((size_t)slot * kQTile + row) * D;
+  float4* part = reinterpret_cast<float4*>(P.ppart_o);
+  {
+    float4* po = part + (size_t)(slot0 + pr.split) * (D / 4) * kQTile + row;
 #pragma unroll
-  for (int cb = 0; cb < D / 32 && !failed; ++cb) {
-    uint32_t ov[32];
-    tmem_ld32(o_col + cb * 32, ov);
-    if (valid) {
+    for (int cb = 0; cb < D / 32 && !failed; ++cb) {
+      uint32_t ov[32];
+      tmem_ld32(o_col + cb * 32, ov);
+      if (valid) {
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        float4 v = make_float4(__uint_as_float(ov[4 * q]) * inv, __uint_as_float(ov[4 * q + 1]) * inv,
-                               __uint_as_float(ov[4 * q + 2]) * inv,
-                               __uint_as_float(ov[4 * q + 3]) * inv);
-        *reinterpret_cast<float4*>(po + cb * 32 + 4 * q) = v;
+        for (int q = 0; q < 8; ++q)
+          po[(size_t)(cb * 8 + q) * kQTile] =
+              make_float4(__uint_as_float(ov[4 * q]) * inv, __uint_as_float(ov[4 * q + 1]) * inv,
+                          __uint_as_float(ov[4 * q + 2]) * inv, __uint_as_float(ov[4 * q + 3]) * inv);
       }
     }
   }
-  if (valid) P.ppart_lse[(size_t)slot * kQTile + row] = lse2 * kLn2;
+  if (valid) P.ppart_lse[(size_t)(slot0 + pr.split) * kQTile + row] = lse2 * kLn2;
   __threadfence();
   asm volatile("bar.sync %0, 128;" ::"r"(bar_id) : "memory");
   if ((tid & 127) == 0) {
@@ -414,17 +417,55 @@ POD_DEV bool prefill_softmax(const Plan& P, const PrefillRange& pr, uint8_t* sm,
     s_flag[i] = (old == R.n_split - 1);
   }
   asm volatile("bar.sync %0, 128;" ::"r"(bar_id) : "memory");
-  if (s_flag[i] && !failed) {
+  if (s_flag[i] && !failed && valid) {
+    // The last split to finish merges all of them, one query row per thread,
+    // always in split order so the result does not depend on which split
+    // finished last: O = sum_s w_s O_s / sum_s w_s, w_s = exp(LSE_s - max LSE).
     __threadfence();
-    const int rows = min(kQTile, R.chunk - qtile * kQTile);
-    const int slot0 = R.slot0 + gidx * R.n_split;
-    const size_t orow0 = (size_t)(R.q_row0 + qtile * kQTile);
-    const int w4 = warp & 3;  // warp w4 of the group merges rows [32 w4, 32 w4 + 32)
-    for (int i0 = w4 * 32; i0 < min(rows, w4 * 32 + 32); i0 += 4)
-      merge_rows_warp<D, 4>(P.ppart_o + (size_t)slot0 * kQTile * D, (long long)kQTile * D, D,
-                            P.ppart_lse + (size_t)slot0 * kQTile, kQTile, 1, R.n_split, i0,
-                            min(rows, w4 * 32 + 32), P.o_p + (orow0 * P.H + head) * D,
-                            (long long)P.H * D, P.lse_p + orow0 * P.H + head, P.H, lane);
+    const int ns = R.n_split;
+    const float* pl = P.ppart_lse + (size_t)slot0 * kQTile + row;
+    float m = -INFINITY;
+    for (int sp = 0; sp < ns; ++sp) m = fmaxf(m, __ldcg(pl + (size_t)sp * kQTile));
+    float wsum = 0.f;
+    for (int sp = 0; sp < ns; ++sp) {
+      const float v = __ldcg(pl + (size_t)sp * kQTile);
+      wsum += (v == -INFINITY) ? 0.f : ex2((v - m) * kLog2e);
+    }
+    const float winv = 1.f / wsum;
+    uint16_t* dst = P.o_p + (out_row * P.H + head) * D;
+    const float4* src = part + (size_t)slot0 * (D / 4) * kQTile + row;
+#pragma unroll 1
+    for (int cb = 0; cb < D / 32; ++cb) {
+      float acc[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) acc[c] = 0.f;
+#pragma unroll 2
+      for (int sp = 0; sp < ns; ++sp) {
+        const float v = __ldcg(pl + (size_t)sp * kQTile);
+        const float w = ((v == -INFINITY) ? 0.f : ex2((v - m) * kLog2e)) * winv;
+        const float4* s4 = src + (size_t)sp * (D / 4) * kQTile + (size_t)(cb * 8) * kQTile;
+        float4 x[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) x[q] = __ldcg(s4 + (size_t)q * kQTile);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          acc[4 * q] = fmaf(w, x[q].x, acc[4 * q]);
+          acc[4 * q + 1] = fmaf(w, x[q].y, acc[4 * q + 1]);
+          acc[4 * q + 2] = fmaf(w, x[q].z, acc[4 * q + 2]);
+          acc[4 * q + 3] = fmaf(w, x[q].w, acc[4 * q + 3]);
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint4 v;
+        v.x = pack_bf16(acc[8 * q + 0], acc[8 * q + 1]);
+        v.y = pack_bf16(acc[8 * q + 2], acc[8 * q + 3]);
+        v.z = pack_bf16(acc[8 * q + 4], acc[8 * q + 5]);
+        v.w = pack_bf16(acc[8 * q + 6], acc[8 * q + 7]);
+        *reinterpret_cast<uint4*>(dst + cb * 32 + 8 * q) = v;
+      }
+    }
+    P.lse_p[out_row * P.H + head] = m + logf(wsum);
   }
   return !failed;
 }

@@ -162,6 +162,8 @@ typedef struct {
   int decode_split_len;      /* keys per decode split                         */
   int ratio_num, ratio_den;  /* prefill share of claims per SM               */
   long long plan_bytes;      /* bytes copied host -> device for the plan      */
+  int prefill_sm_cap;        /* fused CTAs that take prefill work first       */
+  int reserved;
 } pod_plan_info;
 
 /* Per-SM role counts gathered with POD_FLAG_STATS (the "virtual CTA mix"). */

@@ -5,6 +5,8 @@ LSE max-abs <= 1e-3. Scaled-down shapes are compared element by element;
 the full-size configurations (the benchmark's launch configuration) on
 sampled rows the oracle computes one by one.
 """
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -158,17 +160,39 @@ def test_timeout_path_reports_status_and_keeps_results():
     assert pod.close() == pa.POD_OK
 
 
-def test_stats_show_both_roles_per_sm():
-    b = W.make_batch(W.CONFIGS["llama3_8b"])
-    pod = pa.context_for(b, flags=pa.FLAG_STATS)
+def _stats_for(b, policy=None):
+    old = os.environ.get("POD_ATTN_POLICY")
+    if policy:
+        os.environ["POD_ATTN_POLICY"] = policy  # read when the context is created
+    try:
+        pod = pa.context_for(b, flags=pa.FLAG_STATS)
+    finally:
+        if policy:
+            if old is None:
+                del os.environ["POD_ATTN_POLICY"]
+            else:
+                os.environ["POD_ATTN_POLICY"] = old
     db = pa.DeviceBatch(b)
     pre, dec = db.args(pod)
     pod.hybrid(pre, dec, pa.MODE_FUSED)
-    st = pod.stats()
-    plan = pod.last_plan()
+    st, plan = pod.stats(), pod.last_plan()
+    assert pod.close() == pa.POD_OK
+    return st, plan
+
+
+def test_stats_show_both_roles_per_sm():
+    b = W.make_batch(W.CONFIGS["llama3_8b"])
+    # balanced: a decode-heavy batch gives prefill to a subset of the SMs
+    # first; every prefill unit is claimed once and some SMs run both roles
+    st, plan = _stats_for(b, "balanced")
+    assert st["prefill_claims"] == plan["prefill_units"]
+    assert 1 <= plan["prefill_sm_cap"] < plan["num_sms"]
+    assert st["sms_with_both"] >= 1
+    # front (the default): every SM's first claim takes prefill, so most SMs
+    # run both roles
+    st, plan = _stats_for(b)
     assert st["prefill_claims"] == plan["prefill_units"]
     assert st["sms_with_both"] > plan["num_sms"] // 2
-    pod.close()
 
 
 @pytest.mark.slow
