@@ -31,19 +31,21 @@ namespace pod {
 
 // Share of the prefill softmax's exponentials evaluated by exp2_poly on the
 // FMA pipe instead of MUFU (pairs out of 8), and the bf16 packing used for P.
-// Measured on B200 (long-context prefill, 64/8 heads, d 128): 0 pairs with
-// cvt packing is fastest (628 us); 2/3/4 pairs gave 687/717/753 us and integer
-// packing 850 us -- this softmax is bound by issue and latency, not by MUFU.
+// Measured on B200 (long-context prefill, 64/8 heads, d 128, two query tiles
+// per CTA): 0 pairs is fastest; 1/2/3/4 pairs cost 1.3x-1.6x, and replacing
+// every ex2 by a one-cycle stand-in changed nothing, so this softmax is bound
+// by issue and latency (and by the MMA hand-offs), not by MUFU. cvt packing
+// (round to nearest even) is 3 % faster than the integer round-half-away one.
 #ifndef POD_SOFT_EXP2_PAIRS
 #define POD_SOFT_EXP2_PAIRS 0
 #endif
 constexpr int kSoftPairs = POD_SOFT_EXP2_PAIRS;
-#if defined(POD_CVT_PACK)
-#define POD_PACK(a, b) pack_bf16(a, b)
+#if defined(POD_RHA_PACK)
+#define POD_PACK(a, b) pack_bf16_rha(a, b)
 #elif defined(POD_INT_PACK)
 #define POD_PACK(a, b) pack_bf16_int(a, b)
 #else
-#define POD_PACK(a, b) pack_bf16_rha(a, b)
+#define POD_PACK(a, b) pack_bf16(a, b)
 #endif
 
 constexpr float kLog2e = 1.4426950408889634f;
