@@ -99,8 +99,9 @@ struct FusedLayout {
   static constexpr int DEC_ROW = D * 2 + 16;  // padded row: conflict-free ldmatrix
   static constexpr int DEC_STAGE = 2 * kDecTile * DEC_ROW;
   static constexpr int DEC_WARP = kFusedDecStages * DEC_STAGE;
-  static constexpr int DEC_END = kFusedDecWarps * DEC_WARP;
-  static constexpr int DATA_END = PREFILL_END > DEC_END ? PREFILL_END : DEC_END;
+  static constexpr int DEC_END = kFusedDecWarps * DEC_WARP;  // decode turns overlay prefill
+  static constexpr int SIDE_OFF = PREFILL_END > DEC_END ? PREFILL_END : DEC_END;
+  static constexpr int DATA_END = SIDE_OFF + kSideDecWarps * DEC_WARP;  // side decode rings
   static constexpr int BAR_OFF = (DATA_END + 127) & ~127;
   // barrier indices
   static constexpr int B_Q = 0;                         // Q0 and Q1 landed
@@ -113,7 +114,7 @@ struct FusedLayout {
   static constexpr int B_PF = B_SE + 2;                 // P_i in TMEM, one arrival per warp [2]
   static constexpr int B_OR = B_PF + 2;                 // O_i final for the unit [2]
   static constexpr int B_DEC = B_OR + 2;
-  static constexpr int N_BARS = B_DEC + kFusedDecWarps * kFusedDecStages;
+  static constexpr int N_BARS = B_DEC + kFusedWarps * kFusedDecStages;  // a ring per warp
   static constexpr int MISC_OFF = BAR_OFF + N_BARS * 8;
   static constexpr int TOTAL = MISC_OFF + 64;
   static_assert(TOTAL <= 227 * 1024, "fused CTA exceeds the shared memory of an SM");
@@ -528,82 +529,105 @@ __global__ void __launch_bounds__(kFusedThreads, kFusedSlotsPerSm)
   uint32_t last_commit_bar = 0, last_commit_par = 0;
   bool issued_mma = false;
 
-  while (true) {
-    if (tid == 0) {
-      int role = 0, unit = -1;
-      if (!*abort_flag) {
-        // per-SM ticket (SM-aware), or one global counter when that is switched off
-        const int t = atomicAdd(P.sm_ticket + ((P.flags & 0x100) ? 0 : my_sm), 1);
-        const long long num = P.rho_num, den = P.rho_den > 0 ? P.rho_den : 1;
-        bool want_p = ((long long)(t + 1) * num) / den > ((long long)t * num) / den;
-        // front-loaded: each SM's first ticket (one per resident CTA) takes
-        // prefill work, so the long prefill units start first
-        if ((P.flags & 0x200) && t < kFusedSlotsPerSm) want_p = true;
-        // balanced: a fixed set of CTAs (one per SM) serves prefill first and
-        // the rest serve decode first, sized so both finish together
-        if (P.flags & 0x400) want_p = (int)blockIdx.x < P.p_cap;
-        for (int attempt = 0; attempt < 2 && role == 0; ++attempt, want_p = !want_p) {
-          if (want_p && !misc[5]) {
-            const int u = atomicAdd(P.ctl + 0, 1);
-            if (u < P.n_prefill_units) {
-              role = 1;
-              unit = u;
-            } else {
-              misc[5] = 1;
+  // The role warps (softmax, MMA issuer, producer) loop over claims and sync
+  // among themselves on named barrier 1; the side warps stream decode units
+  // from the same queue for the CTA's whole life, so an SM keeps reading
+  // decode K/V while its tensor cores run a prefill unit.
+  auto role_sync = [] { asm volatile("bar.sync 1, %0;" ::"n"(kRoleWarps * 32) : "memory"); };
+  if (warp < kRoleWarps) {
+    while (true) {
+      if (tid == 0) {
+        int role = 0, unit = -1;
+        if (!*abort_flag) {
+          // per-SM ticket (SM-aware), or one global counter when that is switched off
+          const int t = atomicAdd(P.sm_ticket + ((P.flags & 0x100) ? 0 : my_sm), 1);
+          const long long num = P.rho_num, den = P.rho_den > 0 ? P.rho_den : 1;
+          bool want_p = ((long long)(t + 1) * num) / den > ((long long)t * num) / den;
+          // front-loaded: each SM's first ticket (one per resident CTA) takes
+          // prefill work, so the long prefill units start first
+          if ((P.flags & 0x200) && t < kFusedSlotsPerSm) want_p = true;
+          // balanced: a fixed set of CTAs (one per SM) serves prefill first and
+          // the rest serve decode first, sized so both finish together
+          if (P.flags & 0x400) want_p = (int)blockIdx.x < P.p_cap;
+          for (int attempt = 0; attempt < 2 && role == 0; ++attempt, want_p = !want_p) {
+            if (want_p && !misc[5]) {
+              const int u = atomicAdd(P.ctl + 0, 1);
+              if (u < P.n_prefill_units) {
+                role = 1;
+                unit = u;
+              } else {
+                misc[5] = 1;
+              }
+            } else if (!want_p && !misc[6]) {
+              role = 2;  // a decode turn: the warps claim their own units
+              unit = 0;
             }
-          } else if (!want_p && !misc[6]) {
-            role = 2;  // a decode turn: the warps claim their own units
-            unit = 0;
           }
+          if (role && (P.flags & 0x1)) atomicAdd(P.stats + my_sm * 2 + (role - 1), 1);
         }
-        if (role && (P.flags & 0x1)) atomicAdd(P.stats + my_sm * 2 + (role - 1), 1);
+        misc[1] = role;
+        misc[2] = unit;
       }
-      misc[1] = role;
-      misc[2] = unit;
+      role_sync();
+      const int role = misc[1];
+      const int unit = misc[2];
+      if (role == 0) break;
+      if (role == 1) {
+        const PrefillRange pr = prefill_range(P, unit);
+        if (warp < kSoftmaxWarps) {
+          prefill_softmax<D>(P, pr, sm, tmem, ps, tid, abort_flag, misc + 7);
+        } else if (warp == kSoftmaxWarps) {
+          if (lane == 0) {
+            issued_mma = true;
+            prefill_mma<D>(P, pr, sm, tmem, ps, last_commit_bar, last_commit_par, abort_flag);
+          }
+          __syncwarp();
+        } else if (warp == kSoftmaxWarps + 1) {
+          if (lane == 0) prefill_producer<D>(P, T, pr, sm, ps, abort_flag);
+          __syncwarp();
+        }
+        // warps past the producer have no prefill role; they run decode turns
+      } else {
+        // decode turn: every warp is a virtual decode unit runner and claims up
+        // to dec_turn units one at a time; once every prefill unit has been
+        // claimed there is nothing to regroup for, so the warp keeps claiming
+        // until the decode queue is empty. An empty queue ends the turn.
+        for (int k = 0;; ++k) {
+          if (k >= P.dec_turn &&
+              *reinterpret_cast<volatile const int*>(P.ctl + 0) < P.n_prefill_units)
+            break;
+          int u = 0;
+          if (lane == 0) u = atomicAdd(P.ctl + 1, 1);
+          u = __shfl_sync(0xffffffffu, u, 0);
+          if (u >= P.n_decode_units) {
+            if (lane == 0) misc[6] = 1;
+            break;
+          }
+          if (!decode_unit_warp<D, kFusedDecStages>(P, u, sm + warp * L::DEC_WARP,
+                                                    bars + (L::B_DEC + warp * kFusedDecStages) * 8,
+                                                    dec_ring, lane, true, abort_flag))
+            break;
+        }
+      }
+      role_sync();
+      if (*abort_flag) break;
     }
-    __syncthreads();
-    const int role = misc[1];
-    const int unit = misc[2];
-    if (role == 0) break;
-    if (role == 1) {
-      const PrefillRange pr = prefill_range(P, unit);
-      if (warp < kSoftmaxWarps) {
-        prefill_softmax<D>(P, pr, sm, tmem, ps, tid, abort_flag, misc + 7);
-      } else if (warp == kSoftmaxWarps) {
-        if (lane == 0) {
-          issued_mma = true;
-          prefill_mma<D>(P, pr, sm, tmem, ps, last_commit_bar, last_commit_par, abort_flag);
-        }
-        __syncwarp();
-      } else if (warp == kSoftmaxWarps + 1) {
-        if (lane == 0) prefill_producer<D>(P, T, pr, sm, ps, abort_flag);
-        __syncwarp();
+  } else if (allow_decode) {
+    const int sw = warp - kRoleWarps;
+    uint32_t side_ring = 0;
+    while (!*abort_flag) {
+      int u = 0;
+      if (lane == 0) u = atomicAdd(P.ctl + 1, 1);
+      u = __shfl_sync(0xffffffffu, u, 0);
+      if (u >= P.n_decode_units) {
+        if (lane == 0) misc[6] = 1;
+        break;
       }
-      // warps past the producer have no prefill role; they run decode turns
-    } else {
-      // decode turn: every warp is a virtual decode unit runner and claims up
-      // to dec_turn units one at a time; once every prefill unit has been
-      // claimed there is nothing to regroup for, so the warp keeps claiming
-      // until the decode queue is empty. An empty queue ends the turn.
-      for (int k = 0;; ++k) {
-        if (k >= P.dec_turn &&
-            *reinterpret_cast<volatile const int*>(P.ctl + 0) < P.n_prefill_units)
-          break;
-        int u = 0;
-        if (lane == 0) u = atomicAdd(P.ctl + 1, 1);
-        u = __shfl_sync(0xffffffffu, u, 0);
-        if (u >= P.n_decode_units) {
-          if (lane == 0) misc[6] = 1;
-          break;
-        }
-        if (!decode_unit_warp<D, kFusedDecStages>(P, u, sm + warp * L::DEC_WARP,
-                                                  bars + (L::B_DEC + warp * kFusedDecStages) * 8,
-                                                  dec_ring, lane, true, abort_flag))
-          break;
-      }
+      if (!decode_unit_warp<D, kFusedDecStages>(P, u, sm + L::SIDE_OFF + sw * L::DEC_WARP,
+                                                bars + (L::B_DEC + warp * kFusedDecStages) * 8,
+                                                side_ring, lane, true, abort_flag))
+        break;
     }
-    __syncthreads();
-    if (*abort_flag) break;
   }
   // Teardown. After an abort, wait (bounded) for this CTA's own async work.
   if (*abort_flag) {

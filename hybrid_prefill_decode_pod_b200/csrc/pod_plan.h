@@ -19,14 +19,16 @@ constexpr int kQTile = 128;           // prefill query rows per unit (= UMMA M)
 constexpr int kKVTile = 128;          // prefill keys per KV tile (= UMMA N of S)
 constexpr int kPrefillStages = 2;     // K/V smem ring depth in the prefill role
 constexpr int kDecTile = 16;          // decode keys per staged tile (= mma M)
-constexpr int kFusedWarps = 12;       // 8 softmax (2 query tiles) + MMA issuer + TMA producer + 2
-                                      // more decode runners (3 warps per SM sub-partition either way)
+constexpr int kRoleWarps = 10;        // 8 softmax (2 query tiles) + MMA issuer + TMA producer;
+                                      // all of them run decode units in a decode turn
+constexpr int kSideDecWarps = 2;      // warps that stream decode units for the CTA's whole life,
+                                      // beside whatever role the other warps have
+constexpr int kFusedWarps = kRoleWarps + kSideDecWarps;
 constexpr int kFusedThreads = kFusedWarps * 32;
 constexpr int kSoftmaxWarps = 8;
-constexpr int kFusedDecWarps = 12;    // every warp is a virtual decode unit in a decode turn
+constexpr int kFusedDecWarps = kRoleWarps;  // decode runners of a decode turn
 constexpr int kFusedSlotsPerSm = 1;   // persistent CTAs per SM (the CTA owns all TMEM)
-static_assert(kFusedWarps >= kSoftmaxWarps + 2, "softmax warps + MMA issuer + producer");
-static_assert(kFusedDecWarps == kFusedWarps, "a decode turn runs on every warp");
+static_assert(kRoleWarps == kSoftmaxWarps + 2, "softmax warps + MMA issuer + producer");
 constexpr int kFusedDecStages = 2;    // per-warp decode ring depth in the fused kernel
 constexpr int kDecodeWarps = 6;       // warps (virtual decode units) per decode-only CTA
 constexpr int kDecodeStages = 2;      // per-warp ring depth in the decode-only kernel
