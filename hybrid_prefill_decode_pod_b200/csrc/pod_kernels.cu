@@ -593,7 +593,10 @@ __global__ void __launch_bounds__(kFusedThreads, kFusedSlotsPerSm)
         // claimed there is nothing to regroup for, so the warp keeps claiming
         // until the decode queue is empty. An empty queue ends the turn.
         for (int k = 0;; ++k) {
-          if (k >= P.dec_turn &&
+          // balanced: a decode-first CTA stays on decode until the queue is
+          // empty (regrouping after every unit would idle its warps at the
+          // role barrier while the slowest unit finishes)
+          if (k >= P.dec_turn && !(P.flags & 0x400) &&
               *reinterpret_cast<volatile const int*>(P.ctl + 0) < P.n_prefill_units)
             break;
           int u = 0;
