@@ -38,6 +38,10 @@ SHAPES = [
     (4, 4, 128, [(1000, 64)], [2048, 31]),                        # G = 1
     (8, 4, 64, [(129, 129)], [128, 129, 700]),                    # d = 64, G = 2
     (32, 8, 128, [(4096, 512)], [4096] * 4),                      # llama-3-8B rows
+    # G odd: a prefill unit pairs two token tiles of one head (the first tile's
+    # rows meet fully masked KV tiles of the pair's range), with KV splits
+    (6, 2, 128, [(900, 300)], [50, 700]),                         # G = 3, 3 tiles
+    (3, 1, 64, [(1100, 260), (0, 1)], [33]),                      # G = 3, d = 64, 1-token chunk
 ]
 
 
