@@ -2,22 +2,25 @@
 //
 // Roles (POD-Attention §4 "POD-Attention"; the paper's FlashAttention device
 // functions for A100 are prior art here, rebuilt for Blackwell):
-//  * prefill unit: one 128-row query tile of one head against a range of
-//    64-key KV tiles. A TMA producer warp stages Q and K/V (128-byte swizzle),
-//    one thread issues tcgen05.mma (S = Q K^T into TMEM, O += P V into TMEM),
-//    four softmax warps (one thread per query row = TMEM lane) run the online
-//    softmax and write P (bf16) into the K stage the S MMA just consumed.
+//  * prefill unit (pod_prefill.cuh): two 128-row query tiles that share K/V
+//    against a range of 128-key KV tiles. A TMA producer warp stages Q and
+//    K/V (128-byte swizzle), one thread issues tcgen05.mma (S_i = Q_i K^T into
+//    TMEM, O_i += P_i V with P_i read from TMEM), and two groups of four
+//    softmax warps (one thread per query row = TMEM lane) run the online
+//    softmax of the two tiles in ping-pong with the tensor pipe.
 //  * decode unit: one warp (a "virtual decode CTA", paper §4.2.3) streams the
 //    K/V rows of (request, KV head, key split) with TMA bulk copies into a
 //    padded smem ring and runs S^T = K Q^T and O^T += V^T P^T on the legacy
 //    m16n8k16 tensor-core path with the G query heads of the group as N = 8
 //    (the paper's small decode tile, §4.2.1).
 //  * merge: log-sum-exp combination of split partials, in split order.
-//  * fused kernel: persistent CTAs (2 per SM) read %smid, take a ticket from
-//    that SM's counter and pick prefill or decode work in the planned ratio
-//    (§4.1 SM-aware scheduling, §4.4 persistent threads, §5.4.2 proportional
-//    allocation); the last CTA to finish a split group merges it, so no CTA
-//    ever waits for another (the digest's deadlock-free merge requirement).
+//  * fused kernel: one persistent 12-warp CTA per SM. Its ten role warps read
+//    %smid, take a ticket from that SM's counter and pick prefill or decode
+//    work (§4.1 SM-aware scheduling, §4.4 persistent threads, §5.4.2 role
+//    allocation); its two side warps stream decode units for the CTA's whole
+//    life, beside a prefill unit. The last CTA (or warp) to finish a split
+//    group merges it, so no CTA ever waits for another (the digest's
+//    deadlock-free merge requirement).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>

@@ -93,7 +93,7 @@ struct Plan {
 
 // Tensor maps for TMA, passed as a __grid_constant__ kernel parameter.
 // Contiguous layout: k[p] / v[p] map request p's [len, Hk, d] cache with a
-// 64-key box. Paged layout: k[0] / v[0] map the pool as [blocks*16, Hk, d]
+// 128-key box. Paged layout: k[0] / v[0] map the pool as [blocks*16, Hk, d]
 // with a 16-key (one page) box.
 struct TmaDescs {
   CUtensorMap q;

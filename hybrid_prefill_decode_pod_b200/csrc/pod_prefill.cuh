@@ -10,6 +10,7 @@
 //               O_i += P_i V with P_i read from TMEM as the A operand;
 //   warps 0-3   softmax of tile 0, warps 4-7 softmax of tile 1: one thread per
 //               query row (= TMEM lane), 128 keys per KV tile.
+// (Warps 10-11 of the CTA stream decode units meanwhile; see pod_kernels.cu.)
 // TMEM (512 columns): O0 [0,128), O1 [128,256), S0 [256,384), S1 [384,512);
 // P_i (bf16 pairs) is written over the first 64 columns of S_i.
 // MMA order S0 S1 | PV0 S0' | PV1 S1' | ...: while one softmax group works on
