@@ -2,12 +2,13 @@
 // libpod_attn.so. See include/pod_attn.h for the contract.
 //
 // Planner (POD-Attention §4.2.2-§4.2.3 and §5.4): splits the hybrid batch into
-// prefill units (request, head, 128-row query tile, KV split) and decode units
-// (request, KV head, KV split). Prefill KV splits are capped so the prefill
-// units stay within two waves of persistent slots (§4.2.3); the per-SM claim
-// ratio is proportional to the two queues' lengths (§5.4.2). The plan is a
-// pure function of the shapes and the SM count, so FUSED, SERIAL and
-// TWO_STREAM compute bitwise-identical results.
+// prefill units (request, pair of 128-row query tiles sharing K/V, KV split)
+// and decode units (request, KV head, KV split), chooses the split counts, and
+// sets the role policy the fused kernel's per-SM tickets follow (§4.1, §5.4.2).
+// The plan is a pure function of the shapes, the SM count and whether the call
+// is one fused launch (which leaves the prefill unsplit when decodes share it);
+// on a common plan FUSED, SERIAL and TWO_STREAM compute bitwise-identical
+// results.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -532,6 +533,26 @@ int stage_plan(pod_attn_ctx* c, const pod_prefill_args* pa, const pod_decode_arg
   return POD_OK;
 }
 
+// Capacities of the per-call tables and the plan layout, from the config,
+// the head counts and the SM count already set in c.
+void size_context(pod_attn_ctx* c) {
+  const pod_attn_config* cfg = &c->cfg;
+  const int slots = c->num_sms * c->slots_per_sm;
+  const long long qtiles = (long long)cfg->max_prefill_tokens / kQTile + cfg->max_prefill_reqs;
+  c->cap_punits = (int)std::min<long long>(qtiles * c->H * kMaxPrefillSplit, 1 << 24);
+  c->cap_pgroups =
+      (int)std::min<long long>(std::min<long long>(qtiles * c->H, 2LL * slots), 1 << 24);
+  c->cap_pslots = 4 * slots;  // units x splits <= 2 slots, two query tiles per unit
+  c->cap_pgroups = std::max(c->cap_pgroups, 1);
+  c->cap_dreqs = std::max(cfg->max_decode_reqs, 1);
+  c->cap_dunits =
+      (int)std::max<long long>(16LL * c->num_sms * 8, (long long)c->cap_dreqs * c->Hk * 2);
+  c->cap_dgroups = c->cap_dreqs * c->Hk;
+  c->cap_dslots = c->cap_dunits;
+  c->lay = plan_layout(c);
+  c->plan_cap = c->lay.end;
+}
+
 }  // namespace
 
 // =================================================================== C ABI
@@ -608,19 +629,7 @@ int pod_attn_create(pod_attn_ctx** out, const pod_attn_config* cfg) {
   if (decode_occupancy(D, &dec_blocks) != cudaSuccess || dec_blocks < 1) return fail(POD_ECUDA);
   c->decode_grid = c->num_sms * dec_blocks;
 
-  // capacities
-  const int slots = c->num_sms * c->slots_per_sm;
-  const long long qtiles = (long long)cfg->max_prefill_tokens / kQTile + cfg->max_prefill_reqs;
-  c->cap_punits = (int)std::min<long long>(qtiles * H * kMaxPrefillSplit, 1 << 24);
-  c->cap_pgroups = (int)std::min<long long>(std::min<long long>(qtiles * H, 2LL * slots), 1 << 24);
-  c->cap_pslots = 4 * slots;  // units x splits <= 2 slots, two query tiles per unit
-  c->cap_pgroups = std::max(c->cap_pgroups, 1);
-  c->cap_dreqs = std::max(cfg->max_decode_reqs, 1);
-  c->cap_dunits = (int)std::max<long long>(16LL * c->num_sms * 8, (long long)c->cap_dreqs * Hk * 2);
-  c->cap_dgroups = c->cap_dreqs * Hk;
-  c->cap_dslots = c->cap_dunits;
-  c->lay = plan_layout(c);
-  c->plan_cap = c->lay.end;
+  size_context(c);
 
   if (cudaMalloc(&c->d_plan, c->plan_cap) != cudaSuccess) return fail(POD_ENOMEM);
   if (cudaMalloc(&c->d_ppart_o, sizeof(float) * (size_t)c->cap_pslots * kQTile * D) != cudaSuccess)
