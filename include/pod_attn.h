@@ -86,16 +86,20 @@ typedef enum {
 typedef enum { POD_KV_CONTIGUOUS = 0, POD_KV_PAGED = 1 } pod_kv_layout;
 
 /* How pod_attn_hybrid runs the batch.
- * FUSED: one persistent launch; each CTA reads its SM id and takes prefill or
- *   decode work units from per-SM tickets in the planned ratio (POD-Attention
- *   §4.1 "SM-aware CTA Scheduling", §4.4 persistent-thread form, §5.4.2
- *   proportional allocation).
+ * FUSED: one persistent launch, one CTA per SM; the CTA reads its SM id and
+ *   takes prefill or decode work units from per-SM tickets (POD-Attention §4.1
+ *   "SM-aware CTA Scheduling", §4.4 persistent-thread form, §5.4.2 role
+ *   allocation) while two of its warps stream decode units throughout.
  * SERIAL: the prefill-only launch, then the decode launch and the merge
  *   launch, on the caller's stream (the paper's FA_Serial baseline, §2.1/§3).
  * TWO_STREAM: prefill on the caller's stream, decode + merge on an internal
  *   stream, joined back with events (the paper's FA_Streams baseline, §3.2).
- * All three modes use the same work decomposition and merge order, so their
- * outputs are bitwise identical. */
+ * The decode decomposition is the same in all three modes. The prefill KV
+ * split count may differ: a FUSED call that also carries decodes leaves the
+ * prefill unsplit, the other modes split it when that shortens the prefill
+ * launch. Split partials are merged in split order, so on a common plan the
+ * modes' outputs are bitwise identical, and otherwise they differ only by the
+ * rounding of the merge. */
 typedef enum { POD_MODE_FUSED = 0, POD_MODE_SERIAL = 1, POD_MODE_TWO_STREAM = 2 } pod_mode;
 
 /* Flags for pod_attn_config.flags */
@@ -156,7 +160,7 @@ typedef struct {
 typedef struct {
   int num_sms;               /* SMs on the device                             */
   int slots_per_sm;          /* persistent CTAs per SM in the fused launch    */
-  int prefill_units;         /* (request, head, 128-row tile, KV split) units */
+  int prefill_units;         /* (request, pair of 128-row tiles, split) units */
   int prefill_split;         /* KV splits per prefill tile (max over reqs)    */
   int decode_units;          /* (request, KV head, KV split) units            */
   int decode_split_len;      /* keys per decode split                         */
