@@ -84,6 +84,14 @@ PROBE_CONFIGS = {
     "long_context_probe": HybridConfig(
         "long_context_probe", 64, 8, 128, prefill=((4096, 1024),), decode_ctx=(4096,) * 16),
 }
+# Chunked prefill of a 16K-token prompt in chunks of 512 beside 64 decodes at the
+# same context (the paper's per-chunk study of a long prompt, restated on
+# synthetic Llama-3-8B-shaped inputs): point i has prior 512 i and decodes at
+# context 512 (i + 1), i = 0 .. 31.
+for _i in range(32):
+    PROBE_CONFIGS["chunked16k_%d" % _i] = HybridConfig(
+        "chunked16k_%d" % _i, 32, 8, 128, prefill=((512 * _i, 512),),
+        decode_ctx=(512 * (_i + 1),) * 64)
 
 # Human-readable descriptions used in the benchmark's JSON line.
 CONFIG_DESCRIPTIONS = {
@@ -93,6 +101,7 @@ CONFIG_DESCRIPTIONS = {
     "long_context": "long-context 70B-like: 64 q / 8 kv heads, d 128; 1 prefill chunk 1024 after prior 16384 + 16 decodes U[16384, 32768]",
     "paged": "paged-KV: 32 q / 8 kv heads, d 128; 2 prefill chunks of 512 (priors 2048, 8192) + 128 decodes U[1024, 16384], 16-token blocks, permuted",
     "long_context_probe": "profiling probe: 64 q / 8 kv heads, d 128; 1 prefill chunk 1024 after prior 4096 + 16 decodes at 4096",
+    **{"chunked16k_%d" % i: "chunk %d of a 16K prompt: 32 q / 8 kv heads, d 128; prefill chunk 512 after prior %d + 64 decodes at %d" % (i, 512 * i, 512 * (i + 1)) for i in range(32)},
 }
 
 

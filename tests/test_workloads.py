@@ -57,3 +57,15 @@ def test_algorithmic_work_counts():
     assert f_d == 4 * 3
     assert b_p == 2 * 2 * 2 + 2 * 2 * 2 + 2 * 4
     assert b_d == 3 * 2 * 2 + 2 * 2 + 4
+
+
+def test_chunked_16k_sweep_points():
+    """Chunk i of a 16K prompt: prior 512 i, a 512-token chunk, 64 decodes at the
+    context the prompt has reached."""
+    for i in (0, 5, 31):
+        c = W.get_config("chunked16k_%d" % i)
+        assert (c.num_qo_heads, c.num_kv_heads, c.head_dim) == (32, 8, 128)
+        assert c.prefill == ((512 * i, 512),)
+        assert c.decode_ctx == (512 * (i + 1),) * 64
+        assert "chunked16k_%d" % i in W.CONFIG_DESCRIPTIONS
+    assert sum(k.startswith("chunked16k_") for k in W.PROBE_CONFIGS) == 32
