@@ -3,11 +3,14 @@
 One "step" is one ``pod_attn_hybrid`` call (FUSED) on a synthetic hybrid batch
 whose inputs are already resident in HBM; L2 is flushed (a write larger than
 L2) before every timed call and each call is timed with CUDA events on the
-launching stream. The same run also times the library's SERIAL and TWO_STREAM
-modes and the prefill-only / decode-only launches, reports the fused
-max(FLOP, HBM) roofline fraction with the measured peaks, the fp64 oracle on
-the host cores (bounded sample), the clocks seen during the timed region, and
-an end-to-end number through the C ABI with host buffers.
+launching stream. The headline workload is the long-context mix (64 q / 8 kv
+heads, d 128, a 1024-token chunk after 16384 cached tokens plus 16 decodes of
+16K-32K keys). The same run times the library's SERIAL and TWO_STREAM modes
+and the prefill-only / decode-only launches, reports the fused max(FLOP, HBM)
+roofline fraction with the measured peaks, times FUSED / SERIAL / TWO_STREAM
+on the other full-size configurations, times one full fp64 oracle call on the
+host cores, samples the clocks during the timed region, and measures the same
+call end to end through the C ABI with host buffers.
 
 Launch: ``python bench.py --gpus N --steps K --warmup W`` (N > 1 under
 torch.distributed.run: N independent replicas, one per GPU, max over ranks).
@@ -37,7 +40,9 @@ from hybrid_prefill_decode_pod_b200 import workloads as W  # noqa: E402
 
 METRIC = "hybrid attention µs/call & % of max(FLOP,HBM) roofline vs serial P+D, 1 B200"
 UNIT = "us/call"
-DEFAULT_WORKLOAD = "llama3_8b"
+DEFAULT_WORKLOAD = "long_context"
+# the other full-size configurations, timed in the same run as extra keys
+EXTRA_WORKLOADS = ("llama3_8b", "decode_heavy", "paged")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 CSRC = os.path.join(ROOT, "hybrid_prefill_decode_pod_b200", "csrc")
 
@@ -169,67 +174,95 @@ def dist_barrier(world):
 
 
 # ----------------------------------------------------------------- CPU oracle leg
-def oracle_sample_time(batch, budget_s: float, seed: int = 0):
-    """Time the fp64 oracle on a random sample of (row, head) items and scale to
-    one full call by FLOPs. Returns (us_per_call, cores, description)."""
+def oracle_full_call(batch):
+    """One full, unsampled fp64 oracle call on every host core (wall clock).
+    Returns (us, threads)."""
     import oracle
-    cfg = batch.cfg
-    H, d = cfg.num_qo_heads, cfg.head_dim
-    rng = np.random.default_rng(seed)
-    # per-item key counts
-    pk = []
-    for p, c in zip(batch.priors, batch.chunks):
-        pk.append(p + 1 + np.arange(c))
-    pk = np.concatenate(pk) if pk else np.zeros(0, np.int64)
-    dk = np.asarray(batch.ctx, np.int64)
-    total_keys = pk.sum() * H + dk.sum() * H
-    # calibrate: a small sample first
     n_threads = oracle.max_threads()
-    frac = 1e-4
-    spent = 0.0
-    for _ in range(6):
-        np_items = max(1, int(len(pk) * H * frac))
-        nd_items = max(1, int(len(dk) * H * frac)) if len(dk) else 0
-        np_items = min(np_items, len(pk) * H)
-        nd_items = min(nd_items, len(dk) * H)
-        ps = np.sort(rng.choice(len(pk) * H, size=np_items, replace=False)) if len(pk) else None
-        ds = np.sort(rng.choice(len(dk) * H, size=nd_items, replace=False)) if len(dk) else None
+    t0 = time.perf_counter()
+    oracle.hybrid(batch)
+    return (time.perf_counter() - t0) * 1e6, n_threads
+
+
+class OracleSampler:
+    """The oracle on a fixed fraction of a call's (row, head) items, a fresh
+    random sample every step, scaled to one call by key count (the oracle's
+    work is proportional to the keys it visits)."""
+
+    def __init__(self, batch, step_seconds: float):
+        import oracle
+        self.oracle = oracle
+        self.batch = batch
+        H = batch.cfg.num_qo_heads
+        self.H = H
+        pk = [p + 1 + np.arange(c) for p, c in zip(batch.priors, batch.chunks)]
+        self.pk = np.concatenate(pk) if pk else np.zeros(0, np.int64)
+        self.dk = np.asarray(batch.ctx, np.int64)
+        self.total_keys = int(self.pk.sum() * H + self.dk.sum() * H)
+        self.threads = oracle.max_threads()
+        # calibrate the fraction on a small sample so one step takes ~step_seconds
+        self.frac = 1e-3
+        _, dt, keys = self._run(1e-3, seed=12345)
+        per_key = dt / max(keys, 1)
+        self.frac = float(min(1.0, max(1e-4, step_seconds / max(per_key * self.total_keys, 1e-9))))
+
+    def _run(self, frac, seed):
+        # whole rows (every head of a row) keep the oracle's memory access
+        # pattern that of a full call: a random window of prefill rows and a
+        # random subset of decode requests
+        rng = np.random.default_rng(seed)
+        H = self.H
+        n_p, n_d = len(self.pk), len(self.dk)
+        ps = ds = None
+        keys = 0
+        if n_p:
+            w = max(1, int(round(n_p * frac)))
+            r0 = int(rng.integers(0, n_p - w + 1))
+            rows = np.arange(r0, r0 + w)
+            ps = (rows[:, None] * H + np.arange(H)[None, :]).reshape(-1)
+            keys += int(self.pk[rows].sum()) * H
+        if n_d:
+            reqs = np.sort(rng.choice(n_d, size=max(1, int(round(n_d * frac))), replace=False))
+            ds = (reqs[:, None] * H + np.arange(H)[None, :]).reshape(-1)
+            keys += int(self.dk[reqs].sum()) * H
         t0 = time.perf_counter()
-        oracle.hybrid(batch, prefill_sample=ps, decode_sample=ds)
-        dt = time.perf_counter() - t0
-        keys = (pk[ps // H].sum() if ps is not None else 0) + (dk[ds // H].sum() if ds is not None else 0)
-        spent += dt
-        if dt > budget_s * 0.3 or spent > budget_s:
-            break
-        if frac >= 0.25:
-            break
-        frac = min(0.25, frac * max(2.0, min(8.0, budget_s * 0.4 / max(dt, 1e-3))))
-    us = dt / max(keys, 1) * total_keys * 1e6
-    desc = ("%d prefill + %d decode (row, head) items drawn at random (%.3g%% of the keys), "
-            "scaled to one call by key count; fp64, %d OpenMP threads"
-            % (0 if ps is None else len(ps), 0 if ds is None else len(ds),
-               100.0 * keys / total_keys, n_threads))
-    return us, n_threads, desc, dt
+        self.oracle.hybrid(self.batch, prefill_sample=ps, decode_sample=ds)
+        return None, time.perf_counter() - t0, keys
+
+    def step(self, seed):
+        """(us per full call, seconds spent, fraction of the call's keys)."""
+        _, dt, keys = self._run(self.frac, seed)
+        return dt / max(keys, 1) * self.total_keys * 1e6, dt, keys / self.total_keys
+
+    def describe(self, key_frac):
+        return ("each step: the fp64 oracle on a fresh random sample of whole rows (a window of "
+                "%.3g%% of the prefill rows and %.3g%% of the decode requests, every head; %.3g%% "
+                "of the call's key work), timed by wall clock and scaled to one call by key count; "
+                "%d OpenMP threads" % (100 * self.frac, 100 * self.frac, 100 * key_frac,
+                                       self.threads))
 
 
 def run_reference(args, rank, world):
+    """The base contract's reference arm: the fp64 oracle (rank 0 only)."""
     if rank != 0:
         return 0
     batch = W.make_batch(W.get_config(args.workload))
-    vals = []
+    sampler = OracleSampler(batch, args.ref_step_seconds)
+    vals, fracs = [], []
     for i in range(args.warmup + args.steps):
-        budget = 0.5 if i < args.warmup else args.ref_step_seconds
-        us, cores, desc, _ = oracle_sample_time(batch, budget, seed=i)
+        us, _, kf = sampler.step(seed=i)
         if i >= args.warmup:
             vals.append(us)
+            fracs.append(kf)
     v = statistics.median(vals)
+    desc = sampler.describe(statistics.median(fracs))
     line = {
         "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": v / 1000.0,
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
         "config": {"workload": args.workload, "description": W.CONFIG_DESCRIPTIONS[args.workload]},
-        "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+        "cpu_baseline": {"value": v, "unit": UNIT, "cores": sampler.threads, "kind": "oracle",
                          "sample": desc},
         "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -238,7 +271,7 @@ def run_reference(args, rank, world):
 
 
 # ----------------------------------------------------------------- GPU leg
-def time_calls(fn, n, flush_buf, stream, per_call=True):
+def time_calls(fn, n, flush_buf, stream):
     """Time n calls of fn() with CUDA events on `stream`; L2 flushed before each."""
     times = []
     for _ in range(n):
@@ -253,6 +286,57 @@ def time_calls(fn, n, flush_buf, stream, per_call=True):
     return [s.elapsed_time(e) * 1000.0 for s, e in times]  # us
 
 
+def mean(xs):
+    return sum(xs) / len(xs)
+
+
+def roofline_bound(batch, peaks):
+    """Algorithmic FLOPs and bytes of one call and the fused bound
+    T* = max(F / tensor peak, B / HBM peak) in us."""
+    cfg = batch.cfg
+    f_p, f_d, b_p, b_d = W.algorithmic_work(cfg.num_qo_heads, cfg.num_kv_heads, cfg.head_dim,
+                                            batch.priors, batch.chunks, batch.ctx,
+                                            paged=cfg.paged)
+    F, B = f_p + f_d, b_p + b_d
+    t_tc = F / (peaks["bf16_tflops"] * 1e12) * 1e6
+    t_bw = B / (peaks["hbm_gbs"] * 1e9) * 1e6
+    return F, B, max(t_tc, t_bw), ("tensor" if t_tc > t_bw else "hbm"), f_p
+
+
+def time_modes(pa, pod, pre, dec, stream, flush, steps, warmup):
+    """Mean us of FUSED, SERIAL and TWO_STREAM calls (warm-up first)."""
+    out = {}
+    for name, mode in (("fused", pa.MODE_FUSED), ("serial", pa.MODE_SERIAL),
+                       ("two_stream", pa.MODE_TWO_STREAM)):
+        fn = (lambda m: (lambda: pod.hybrid(pre, dec, m, stream)))(mode)
+        for _ in range(warmup):
+            fn()
+        out[name] = mean(time_calls(fn, steps, flush, stream))
+    return out
+
+
+def run_extra_workload(pa, name, dev, local, stream, flush, peaks, steps):
+    """FUSED / SERIAL / TWO_STREAM on another full-size configuration."""
+    batch = W.make_batch(W.CONFIGS[name])
+    pod = pa.context_for(batch, device=local)
+    db = pa.DeviceBatch(batch, device=dev)
+    pre, dec = db.args(pod)
+    t = time_modes(pa, pod, pre, dec, stream, flush, steps, 3)
+    st = pod.status(stream)
+    plan = pod.last_plan()
+    pod.close()
+    if st != pa.POD_OK:
+        raise RuntimeError("device status %d on %s" % (st, name))
+    F, B, t_star, bound, _ = roofline_bound(batch, peaks)
+    del db
+    torch.cuda.empty_cache()
+    return {"fused_us": t["fused"], "serial_us": t["serial"], "two_stream_us": t["two_stream"],
+            "t_star_us": t_star, "bound": bound, "fused_roofline_frac": t_star / t["fused"],
+            "speedup_vs_serial": t["serial"] / t["fused"],
+            "speedup_vs_two_stream": t["two_stream"] / t["fused"], "steps": steps,
+            "decode_split_len": plan["decode_split_len"], "prefill_units": plan["prefill_units"]}
+
+
 def run_gpu(args, rank, world, local):
     from hybrid_prefill_decode_pod_b200 import pod_attn as pa
     dev = torch.device("cuda", local)
@@ -260,22 +344,13 @@ def run_gpu(args, rank, world, local):
     peaks, peak_kind = load_peaks()
     cfg = W.get_config(args.workload)
     batch = W.make_batch(cfg)
-    paged = cfg.paged
     pod = pa.context_for(batch, device=local, flags=pa.FLAG_STATS if args.stats else 0)
     db = pa.DeviceBatch(batch, device=dev)
     pre, dec = db.args(pod)
     stream = torch.cuda.current_stream(dev)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device=dev)
-
-    H, Hk, d = cfg.num_qo_heads, cfg.num_kv_heads, cfg.head_dim
-    f_p, f_d, b_p, b_d = W.algorithmic_work(H, Hk, d, batch.priors, batch.chunks, batch.ctx,
-                                            paged=paged)
-    F, B = f_p + f_d, b_p + b_d
-    tc_peak = peaks["bf16_tflops"] * 1e12
-    bw_peak = peaks["hbm_gbs"] * 1e9
-    t_star = max(F / tc_peak, B / bw_peak) * 1e6  # us
-    bound = "tensor" if F / tc_peak > B / bw_peak else "hbm"
+    F, B, t_star, bound, f_prefill = roofline_bound(batch, peaks)
 
     def call(mode):
         return lambda: pod.hybrid(pre, dec, mode, stream)
@@ -294,7 +369,8 @@ def run_gpu(args, rank, world, local):
         pod.close()
         if rank == 0:
             print(json.dumps({"only": args.only, "workload": args.workload,
-                              "us_median": statistics.median(ts), "status": st}), flush=True)
+                              "us_mean": mean(ts), "us_median": statistics.median(ts),
+                              "status": st}), flush=True)
         return 0 if st == pa.POD_OK else 1
 
     # warm-up (>= 3)
@@ -316,9 +392,8 @@ def run_gpu(args, rank, world, local):
     torch.cuda.synchronize()
     dist_barrier(world)
     clocks = clk.summary()
-    fused_mean = sum(fused) / len(fused)
-    fused_med = statistics.median(fused)
-    fused_max_ranks = dist_max(fused_mean, world)
+    fused_mean = mean(fused)
+    value = dist_max(fused_mean, world)
 
     # ---- the library's own baselines and the standalone phases (same run)
     extra_steps = max(5, args.steps // 2)
@@ -326,7 +401,6 @@ def run_gpu(args, rank, world, local):
     two = time_calls(call(pa.MODE_TWO_STREAM), extra_steps, flush, stream)
     p_only = time_calls(lambda: pod.prefill_only(pre, stream), extra_steps, flush, stream) if pre else [0.0]
     d_only = time_calls(lambda: pod.decode_only(dec, stream), extra_steps, flush, stream) if dec else [0.0]
-    plan = None
     pod.hybrid(pre, dec, pa.MODE_FUSED, stream)
     plan = pod.last_plan()
     stats = pod.stats(stream) if args.stats else None
@@ -338,47 +412,62 @@ def run_gpu(args, rank, world, local):
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(pa, pod, batch, db, dev, stream, min(args.steps, args.e2e_steps), flush)
+    pod.close()
+    del db
+    torch.cuda.empty_cache()
 
-    # ---- CPU oracle baseline (rank 0, N = 1 only)
+    # ---- the other full-size configurations (single GPU only)
+    extras = {}
+    if world == 1 and not args.no_extras:
+        for name in EXTRA_WORKLOADS:
+            if name != args.workload:
+                extras[name] = run_extra_workload(pa, name, dev, local, stream, flush, peaks,
+                                                  args.extra_steps)
+
+    # ---- CPU oracle baseline: one full call (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
-        us, cores, desc, _ = oracle_sample_time(batch, args.cpu_seconds)
-        cpu = {"value": us, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
+        us, cores = oracle_full_call(batch)
+        cpu = {"value": us, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": "one full, unsampled call of this workload (every (row, head) item), "
+                         "wall clock, fp64, %d OpenMP threads" % cores}
 
-    achieved_tflops = F / (fused_med * 1e-6) / 1e12
-    achieved_gbs = B / (fused_med * 1e-6) / 1e9
+    achieved_tflops = F / (value * 1e-6) / 1e12
+    achieved_gbs = B / (value * 1e-6) / 1e9
     if bound == "hbm":
         roof = {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": achieved_gbs / peaks["hbm_gbs"]}
     else:
         roof = {"bound": "tensor", "achieved": achieved_tflops, "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": achieved_tflops / peaks["bf16_tflops"]}
-    roof["peak_kind"] = peak_kind + " (burst)"
+    roof["peak_kind"] = ("of measured" if peak_kind == "measured" else "of fallback") + " (burst)"
     roof["kernel"] = "pod_fused_kernel"
     roof["traffic"] = committed_traffic(args.workload)
     roof["algorithmic_bytes"] = B
     roof["algorithmic_flops"] = F
+    roof["statistic"] = "mean of the timed calls (the same as value)"
 
-    med = statistics.median
     line = {
-        "metric": METRIC, "value": fused_max_ranks, "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": fused_max_ranks / 1000.0,
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": value / 1000.0,
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "config": {"workload": args.workload, "description": W.CONFIG_DESCRIPTIONS[args.workload],
                    "l2": "flushed before every timed call (write of %d MB)" % (flush.numel() * 4 >> 20),
                    "mode": "fused", "parallelism": "replicas" if world > 1 else "single GPU"},
         "roofline": roof,
-        "fused_roofline_frac": t_star / fused_med,
+        "fused_roofline_frac": t_star / value,
         "t_star_us": t_star,
-        "fused_us": {"mean": fused_mean, "median": fused_med, "p10": float(np.percentile(fused, 10)),
-                     "p90": float(np.percentile(fused, 90))},
-        "serial_us": med(serial), "two_stream_us": med(two),
-        "prefill_only_us": med(p_only), "decode_only_us": med(d_only),
-        "speedup_vs_serial": med(serial) / fused_med,
-        "speedup_vs_two_stream": med(two) / fused_med,
+        "fused_us": {"mean": fused_mean, "median": statistics.median(fused),
+                     "p10": float(np.percentile(fused, 10)), "p90": float(np.percentile(fused, 90))},
+        "serial_us": mean(serial), "two_stream_us": mean(two),
+        "prefill_only_us": mean(p_only), "decode_only_us": mean(d_only),
+        "prefill_only_tflops": f_prefill / (mean(p_only) * 1e-6) / 1e12 if pre else None,
+        "speedup_vs_serial": mean(serial) / fused_mean,
+        "speedup_vs_two_stream": mean(two) / fused_mean,
         "tflops": achieved_tflops, "gbs": achieved_gbs,
         "plan": plan,
+        "other_workloads": extras,
         "clocks": clocks,
         "gpu_launches": args.steps,
         "wall_s_timed_region": wall,
@@ -387,7 +476,6 @@ def run_gpu(args, rank, world, local):
     }
     if stats:
         line["virtual_cta_mix"] = stats
-    pod.close()
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
@@ -425,7 +513,7 @@ def run_e2e(pa, pod, batch, db, dev, stream, steps, flush):
         e.record(stream)
         e.synchronize()
         times.append(s.elapsed_time(e) * 1000.0)
-    return {"value": statistics.median(times), "unit": UNIT, "h2d_bytes_per_step": h2d,
+    return {"value": mean(times), "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": steps,
             "note": "inputs (Q and every K/V byte the call reads) copied from pinned host memory each step"}
 
@@ -437,11 +525,13 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.CONFIGS) + sorted(W.PROBE_CONFIGS))
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-step-seconds", type=float, default=2.0)
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the other full-size configurations")
+    ap.add_argument("--extra-steps", type=int, default=10)
     ap.add_argument("--stats", action="store_true")
     ap.add_argument("--only", default=None,
                     choices=["fused", "serial", "two_stream", "prefill_only", "decode_only"],

@@ -430,8 +430,8 @@ int build_plan(pod_attn_ctx* c, const pod_prefill_args* pa, const pod_decode_arg
   Q.paged = paged ? 1 : 0;
   Q.bt_stride_p = (np && paged) ? pa->block_table_stride : 0;
   Q.bt_stride_d = (nd && paged) ? da->block_table_stride : 0;
-  Q.flags = (int)c->cfg.flags | (c->smid_aware ? 0 : 0x100) | (c->policy == 4 ? 0x200 : 0) |
-            (c->policy == 5 ? 0x400 : 0);
+  Q.flags = (int)c->cfg.flags | (c->smid_aware ? 0 : kFlagGlobalTicket) | (c->policy == 4 ? kFlagFrontPolicy : 0) |
+            (c->policy == 5 ? kFlagBalancedPolicy : 0);
   Q.p_cap = p_cap;
   Q.dec_turn = c->dec_turn;
   Q.wait_budget = kDefaultWaitBudget;

@@ -543,15 +543,15 @@ __global__ void __launch_bounds__(kFusedThreads, kFusedSlotsPerSm)
         int role = 0, unit = -1;
         if (!*abort_flag) {
           // per-SM ticket (SM-aware), or one global counter when that is switched off
-          const int t = atomicAdd(P.sm_ticket + ((P.flags & 0x100) ? 0 : my_sm), 1);
+          const int t = atomicAdd(P.sm_ticket + ((P.flags & kFlagGlobalTicket) ? 0 : my_sm), 1);
           const long long num = P.rho_num, den = P.rho_den > 0 ? P.rho_den : 1;
           bool want_p = ((long long)(t + 1) * num) / den > ((long long)t * num) / den;
           // front-loaded: each SM's first ticket (one per resident CTA) takes
           // prefill work, so the long prefill units start first
-          if ((P.flags & 0x200) && t < kFusedSlotsPerSm) want_p = true;
+          if ((P.flags & kFlagFrontPolicy) && t < kFusedSlotsPerSm) want_p = true;
           // balanced: a fixed set of CTAs (one per SM) serves prefill first and
           // the rest serve decode first, sized so both finish together
-          if (P.flags & 0x400) want_p = (int)blockIdx.x < P.p_cap;
+          if (P.flags & kFlagBalancedPolicy) want_p = (int)blockIdx.x < P.p_cap;
           for (int attempt = 0; attempt < 2 && role == 0; ++attempt, want_p = !want_p) {
             if (want_p && !misc[5]) {
               const int u = atomicAdd(P.ctl + 0, 1);
@@ -599,7 +599,7 @@ __global__ void __launch_bounds__(kFusedThreads, kFusedSlotsPerSm)
           // balanced: a decode-first CTA stays on decode until the queue is
           // empty (regrouping after every unit would idle its warps at the
           // role barrier while the slowest unit finishes)
-          if (k >= P.dec_turn && !(P.flags & 0x400) &&
+          if (k >= P.dec_turn && !(P.flags & kFlagBalancedPolicy) &&
               *reinterpret_cast<volatile const int*>(P.ctl + 0) < P.n_prefill_units)
             break;
           int u = 0;
@@ -682,12 +682,21 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
 }
 
 // One warp per (decode request, KV head) group whose KV range was split.
+// With kFlagPoisonOnStatus set, a non-zero status word (a decode warp gave up
+// on a bounded wait) makes every group write NaN instead, so a call whose
+// partial results are incomplete cannot be mistaken for a result.
 template <int D>
 __global__ void __launch_bounds__(128) pod_merge_kernel(const __grid_constant__ Plan P) {
   const int gw = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (gw >= P.n_decode_reqs * P.Hk) return;
   const int r = gw / P.Hk, g = gw - (gw / P.Hk) * P.Hk;
+  if ((P.flags & kFlagPoisonOnStatus) && *reinterpret_cast<volatile const int*>(P.status) != 0) {
+    uint16_t* o = P.o_d + ((size_t)r * P.H + (size_t)g * P.G) * D;
+    for (int i = lane; i < P.G * D; i += 32) o[i] = 0x7FC0u;  // bf16 quiet NaN
+    if (lane < P.G) P.lse_d[(size_t)r * P.H + (size_t)g * P.G + lane] = __int_as_float(0x7FC00000);
+    return;
+  }
   const DecodeReq R = P.dreq[r];
   if (R.n_split <= 1) return;
   merge_decode_group<D>(P, R, r, g, lane);

@@ -36,6 +36,12 @@ constexpr int kMaxGroup = 8;          // query heads per KV head (mma N = 8)
 constexpr int kTmemCols = 512;        // TMEM columns per CTA: O0, O1, S0, S1 (128 each)
 constexpr int kMaxSmid = 256;         // per-SM ticket slots (indexed by %smid)
 constexpr long long kDefaultWaitBudget = 2000000000LL;  // cycles (~1 s at 2 GHz)
+// Plan::flags bits set by the library itself (the low byte carries the
+// POD_FLAG_* bits of the context's configuration).
+constexpr int kFlagGlobalTicket = 0x100;    // one ticket counter instead of one per SM
+constexpr int kFlagFrontPolicy = 0x200;     // each SM's first ticket takes prefill
+constexpr int kFlagBalancedPolicy = 0x400;  // a fixed set of CTAs takes prefill first
+constexpr int kFlagPoisonOnStatus = 0x800;  // merge writes NaN when the status word is set
 
 struct PrefillReq {
   int prior, chunk, q_row0, n_qtiles;

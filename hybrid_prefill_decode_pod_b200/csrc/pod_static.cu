@@ -13,7 +13,8 @@
 // The array lives in every GPU that loads the library until the process
 // exits. Every call uses the same array and leaves its contents behind; each
 // call re-initialises what must start at zero. Two calls that overlap on the
-// GPU (different streams, or different host threads) race on it.
+// GPU (different streams, or different host threads) race on it. A call whose
+// decode warps gave up on a bounded device wait writes NaN to its outputs.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -51,7 +52,14 @@ constexpr size_t kLseOff = (kHeadBytes + 255) / 256 * 256;
 constexpr size_t kPartOff = kLseOff + sizeof(float) * kMaxUnits * kMaxGroup;
 constexpr size_t kScratchBytes = kPartOff + sizeof(float) * kMaxUnits * kMaxGroup * kMaxDim;
 
-__device__ __align__(256) unsigned char g_decode_scratch[kScratchBytes];
+}  // namespace
+
+// The scratch array itself: file scope, internal linkage. In host code its
+// name is only a stand-in for the symbol; the device address comes from
+// cudaGetSymbolAddress (setup_device below).
+static __device__ __align__(256) unsigned char g_decode_scratch[kScratchBytes];
+
+namespace {
 
 // Host staging for the head part (copied with one cudaMemcpyAsync per call).
 unsigned char g_host_head[kHeadBytes];
@@ -134,6 +142,14 @@ extern "C" POD_API int pod_attn_decode_static(int num_qo_heads, int num_kv_heads
   };
   while (units_for(split_len) > kMaxUnits) split_len *= 2;  // ends: num_reqs * Hk <= max units
 
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // The per-call plan is copied from one shared host buffer that the next
+  // call overwrites, so a captured copy would replay whatever plan the latest
+  // call left there: refuse while the stream is being captured.
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cap) != cudaSuccess) return POD_ECUDA;
+  if (cap != cudaStreamCaptureStatusNone) return POD_EUNSUPPORTED;
+
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return POD_ECUDA;
   DeviceState* st = nullptr;
@@ -166,7 +182,6 @@ extern "C" POD_API int pod_attn_decode_static(int num_qo_heads, int num_kv_heads
     n_units += R.n_split * Hk;
   }
   const size_t head_bytes = kUnitOff + sizeof(int) * (size_t)n_units;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaMemcpyAsync(st->scratch, g_host_head, head_bytes, cudaMemcpyHostToDevice, s) !=
       cudaSuccess)
     return POD_ECUDA;
@@ -185,6 +200,11 @@ extern "C" POD_API int pod_attn_decode_static(int num_qo_heads, int num_kv_heads
   P.bt_stride_d = paged ? a->block_table_stride : 0;
   P.pool_blocks = paged ? (int)(a->pool_blocks < (1LL << 30) ? a->pool_blocks : (1LL << 30)) : 0;
   P.wait_budget = kDefaultWaitBudget;
+  // The status word lives in the zeroed head of the array: if a decode warp
+  // gives up on a bounded wait in this call, the merge launch writes NaN to
+  // every output row instead of merging partials that are incomplete or left
+  // over from an earlier call.
+  P.flags = kFlagPoisonOnStatus;
   P.dreq = reinterpret_cast<const DecodeReq*>(st->scratch + kReqOff);
   P.dunit_req = reinterpret_cast<const int*>(st->scratch + kUnitOff);
   P.q_d = static_cast<const uint16_t*>(a->q);

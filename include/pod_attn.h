@@ -240,9 +240,12 @@ POD_API int pod_attn_destroy(pod_attn_ctx* ctx);
  * contents behind (each call re-initialises what must start at zero), so
  * calls that overlap on the GPU -- on different streams or from different
  * host threads -- race on it and must not be issued. The copy of the small
- * per-call plan comes from pageable host memory, so the call does not return
- * before the stream has reached it. A device-side wait that runs out is not
- * reported by this entry point (it has no context to hold a status word).
+ * per-call plan comes from one pageable host buffer that the next call
+ * overwrites, so the call does not return before the stream has reached it,
+ * and while `stream` is being captured the call returns POD_EUNSUPPORTED
+ * without enqueuing anything. If a device-side wait runs out, the call has
+ * no context to hold a status word: it writes NaN to every O and LSE element
+ * of the batch instead of a result.
  * ------------------------------------------------------------------------- */
 #define POD_STATIC_MAX_DECODE_REQS 512
 #define POD_STATIC_MAX_KV_HEADS 16

@@ -89,3 +89,22 @@ def test_missing_library_fails_loudly(tmp_path):
             pa.load_library(str(tmp_path / "nope.so"))
         finally:
             pa._lib = pa._lib_backup
+
+
+def test_static_decode_refuses_oversize_batches_on_host(lib):
+    """pod_attn_decode_static checks its fixed array's limits before any CUDA
+    call: more (request, KV head) pairs than its unit table holds, too many
+    requests, too many KV heads."""
+    ctx = (ctypes.c_int * 600)(*([100] * 600))
+    a = pa.DecodeArgs()
+    a.ctx_lens = ctypes.cast(ctx, ctypes.POINTER(ctypes.c_int))
+    a.num_reqs = 300            # 300 x 16 KV heads = 4800 > 4096 units
+    assert lib.pod_attn_decode_static(16, 16, 64, 0, ctypes.byref(a), None) == pa.POD_ECAPACITY
+    a.num_reqs = 513            # more requests than the request table holds
+    assert lib.pod_attn_decode_static(8, 2, 128, 0, ctypes.byref(a), None) == pa.POD_ECAPACITY
+    a.num_reqs = 4              # 32 KV heads > 16
+    assert lib.pod_attn_decode_static(32, 32, 128, 0, ctypes.byref(a), None) == pa.POD_ECAPACITY
+    a.num_reqs = -1
+    assert lib.pod_attn_decode_static(8, 2, 128, 0, ctypes.byref(a), None) == pa.POD_EINVAL
+    assert lib.pod_attn_decode_static(8, 2, 96, 0, ctypes.byref(a), None) == pa.POD_EUNSUPPORTED
+    assert lib.pod_attn_decode_static(8, 2, 128, 0, None, None) == pa.POD_EINVAL

@@ -1,9 +1,9 @@
 """GPU parity: the CUDA path through the C ABI against the fp64 oracle.
 
 Tolerances (bf16 outputs vs fp64): O max-abs <= 1e-2 and relative L2 <= 5e-3;
-LSE max-abs <= 1e-3. Scaled-down shapes are compared element by element;
-the full-size configurations (the benchmark's launch configuration) on
-sampled rows the oracle computes one by one.
+LSE max-abs <= 1e-3. Every output element is compared, on scaled-down shapes
+that span several tiles with ragged tails and on the five full-size
+configurations in the launch configuration the benchmark times.
 """
 import contextlib
 import os
@@ -16,7 +16,7 @@ import oracle
 from hybrid_prefill_decode_pod_b200 import workloads as W
 from hybrid_prefill_decode_pod_b200 import pod_attn as pa
 
-from gpu_util import bitwise_equal, compare, run, sample_indices
+from gpu_util import bitwise_equal, compare, run
 
 pytestmark = pytest.mark.gpu
 
@@ -113,9 +113,10 @@ def test_invariants_on_gpu():
     for r, L in enumerate(b.ctx):
         assert np.abs(out["decode_lse"][r].numpy() - np.log(L)).max() < 1e-5
     t = np.arange(150)
-    # prefill evaluates 3/8 of its exponentials with a polynomial whose relative
-    # error is below 7.5e-5 (csrc/pod_exp2.cuh), which bounds the LSE error here
-    assert np.abs(out["prefill_lse"].numpy() - np.log(t + 1)[:, None]).max() < 1e-4
+    # every score is 0, so every weight is exactly 1 and the row sum is the
+    # exact key count: the LSE differs from ln(count) only by the rounding of
+    # the final log
+    assert np.abs(out["prefill_lse"].numpy() - np.log(t + 1)[:, None]).max() < 1e-5
     # single key: decode L = 1 returns V0 bitwise
     b2 = W.make_custom(8, 2, 128, [], [1, 1], seed=23)
     out2, _ = run(b2, "fused")
@@ -214,17 +215,30 @@ def test_stats_show_both_roles_per_sm():
     assert st["sms_with_both"] >= min(plan["prefill_units"], plan["num_sms"]) // 2
 
 
+_FULL_REF = {}
+
+
+def _full_ref(name):
+    """Batch and full fp64 oracle outputs of a full-size configuration (cached
+    per test session: the oracle is the expensive side)."""
+    if name not in _FULL_REF:
+        _FULL_REF.clear()  # keep one configuration's tensors alive at a time
+        b = W.make_batch(W.CONFIGS[name])
+        _FULL_REF[name] = (b, oracle.hybrid(b))
+    return _FULL_REF[name]
+
+
+FULL_SIZE = [("llama3_8b", "fused"), ("decode_heavy", "fused"),
+             ("long_context", "fused"), ("long_context", "serial"), ("long_context", "two_stream"),
+             ("paged", "fused"), ("paged", "serial"), ("paged", "two_stream")]
+
+
 @pytest.mark.slow
-@pytest.mark.parametrize("name", ["llama3_8b", "decode_heavy", "long_context", "paged"])
-def test_full_size_configs_sampled(name):
-    """Full-size configuration, FUSED launch as benchmarked; oracle on sampled rows."""
-    b = W.make_batch(W.CONFIGS[name])
-    H = b.cfg.num_qo_heads
-    ps = sample_indices(b.total_prefill_tokens, H, 192, 1)
-    ds = sample_indices(b.num_decodes, H, 192, 2)
-    ref = oracle.hybrid(b, prefill_sample=ps, decode_sample=ds)
-    out, plan = run(b, "fused")
-    compare(ref, out, sample={"prefill": ps, "decode": ds})
-    # properties at any size: finite everywhere, LSE >= max score bound sanity
-    for k in ("prefill_o", "decode_o", "prefill_lse", "decode_lse"):
-        assert torch.isfinite(out[k].float()).all(), k
+@pytest.mark.parametrize("name,mode", FULL_SIZE)
+def test_full_size_configs_every_element(name, mode):
+    """Full-size configuration in the launch configuration the benchmark times,
+    every output element against the fp64 oracle. SERIAL and TWO_STREAM take
+    their own prefill plans (they may split the KV range where FUSED does not)."""
+    b, ref = _full_ref(name)
+    out, plan = run(b, mode)
+    compare(ref, out)

@@ -3,9 +3,10 @@
 It exists for callers whose device memory is all owned by someone else (an
 engine that reserves HBM for its KV cache up front, a plugin handed its
 buffers by a host framework) and so cannot cudaMalloc when they call
-attention. Its output must agree with the context-based pod_attn_decode_only
-at the parity tolerances, on two calls in a row (the second call reuses the
-library's scratch array the first one left behind).
+attention. Each case checks its output against the fp64 oracle at the parity
+tolerances and against the context-based pod_attn_decode_only, on two calls in
+a row (the second call reuses the library's scratch array the first one left
+behind), and a batch of another shape runs right after a large one.
 
 This file is collected last so that a run that stops at its first failure has
 already run every other test; it also passes when run alone.
@@ -14,41 +15,62 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from hybrid_prefill_decode_pod_b200 import pod_attn as pa
 from hybrid_prefill_decode_pod_b200 import workloads as W
 
-from gpu_util import LSE_MAX_ABS, O_MAX_ABS, O_REL_L2
+from gpu_util import compare
 
 pytestmark = pytest.mark.gpu
 
 
-def _close(o, lse, o_ref, lse_ref):
-    o, o_ref = o.float().cpu().double(), o_ref.float().cpu().double()
-    assert torch.isfinite(o).all() and torch.isfinite(lse).all()
-    assert (o - o_ref).abs().max().item() <= O_MAX_ABS
-    assert (torch.linalg.norm(o - o_ref) / torch.linalg.norm(o_ref)).item() <= O_REL_L2
-    assert (lse.cpu().double() - lse_ref.cpu().double()).abs().max().item() <= LSE_MAX_ABS
-
-
-@pytest.mark.parametrize("paged", [False, True])
-def test_static_decode_matches_decode_only_twice(paged):
-    # splits and single-split requests, G = 4, contexts with ragged tails
-    b = W.make_custom(32, 8, 128, [], [4096, 1, 700, 5000, 9000, 513, 2048, 77], seed=61,
-                      paged=paged)
+def _static_twice(b, paged):
+    """Two pod_attn_decode_static calls on `b`; each compared with the oracle
+    and with pod_attn_decode_only on the same inputs."""
+    cfg = b.cfg
+    ref = oracle.hybrid(b)
     pod = pa.context_for(b, paged=paged)
     db = pa.DeviceBatch(b, paged=paged)
     _, dec = db.args(pod)
     pod.decode_only(dec)
     assert pod.status() == pa.POD_OK
-    ref_o, ref_lse = db.o_d.clone(), db.lse_d.clone()
-    cfg = b.cfg
+    ctx_o, ctx_lse = db.o_d.clone(), db.lse_d.clone()
     for _ in range(2):
         db.o_d.fill_(float("nan"))
         db.lse_d.fill_(float("nan"))
         pa.decode_static(cfg.num_qo_heads, cfg.num_kv_heads, cfg.head_dim, dec, paged=paged)
         torch.cuda.synchronize()
-        _close(db.o_d, db.lse_d, ref_o, ref_lse)
+        out = {"decode_o": db.o_d.cpu(), "decode_lse": db.lse_d.cpu()}
+        compare(ref, out, keys=("decode",))
+        ctx = {"decode_o": ctx_o.cpu(), "decode_lse": ctx_lse.cpu()}
+        compare({"decode_o": ctx["decode_o"].double().numpy(),
+                 "decode_lse": ctx["decode_lse"].double().numpy()}, out, keys=("decode",))
     assert pod.close() == pa.POD_OK
+
+
+@pytest.mark.parametrize("paged", [False, True])
+def test_static_decode_g4_d128_matches_oracle_twice(paged):
+    # split and single-split requests, G = 4, contexts with ragged tails
+    b = W.make_custom(32, 8, 128, [], [4096, 1, 700, 5000, 9000, 513, 2048, 77], seed=61,
+                      paged=paged)
+    _static_twice(b, paged)
+
+
+def test_static_decode_g8_d64_matches_oracle_twice():
+    b = W.make_custom(64, 8, 64, [], [3000, 17, 1024, 6001, 2], seed=67)
+    _static_twice(b, False)
+
+
+def test_static_decode_split_growth_then_smaller_batch():
+    # 190 short + 10 long requests with 16 KV heads: at 512 keys per split the
+    # units exceed the array's 4096, so the split length grows (to 4096 keys);
+    # the long requests still split 5 ways. A smaller batch of another shape
+    # then reuses the array the large one left behind.
+    ctx = [600] * 190 + [20000] * 10
+    big = W.make_custom(16, 16, 64, [], ctx, seed=71)
+    _static_twice(big, False)
+    small = W.make_custom(16, 4, 128, [], [900, 5, 3333], seed=73)
+    _static_twice(small, False)
 
 
 def test_static_decode_rejects_sizes_beyond_its_array():
