@@ -18,6 +18,7 @@
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
+#include <functional>
 #include <new>
 #include <vector>
 
@@ -33,6 +34,9 @@ cudaError_t launch_fused(const Plan& P, const TmaDescs& T, int grid, int allow_p
 cudaError_t launch_decode(const Plan& P, int max_grid, cudaStream_t s);
 cudaError_t decode_occupancy(int D, int* blocks_per_sm);
 cudaError_t launch_merge(const Plan& P, cudaStream_t s);
+cudaError_t pair_max_clusters(int* clusters);
+cudaError_t launch_fused_pair(const Plan& P, const TmaDescs& T, int grid, int allow_prefill,
+                              int allow_decode, cudaStream_t s);
 }  // namespace pod
 
 using namespace pod;
@@ -59,10 +63,15 @@ struct DeviceGuard {
   }
 };
 
-// Byte offsets of one plan inside the plan buffer (host slot and device copy
-// have the same layout). Everything before `tables` is zeroed each call.
+// Capacity layout of the plan buffer: its size bounds any call's plan. A call
+// packs its plan from the start of the buffer (control words, tickets, stats,
+// merge counters, then the tables it uses) and copies only that much; the
+// control words, tickets, stats and merge counters (everything before the
+// tables) start at zero.
 struct PlanLayout {
-  size_t ctl, ticket, stats, pgroup, dgroup, tables, preq, punits, dreq, dunit, end;
+  size_t ctl, ticket, stats, tables0;                        // fixed part
+  size_t pgroup, dgroup, tables, preq, punits, dreq, dunit;  // capacities
+  size_t end;
 };
 
 }  // namespace
@@ -79,6 +88,9 @@ struct pod_attn_ctx {
   int dec_turn = 1;      // decode units each warp claims per decode turn of a fused CTA
   int dec_split = 0;     // 0: cost model; else keys per decode split (multiple of 16)
   int pre_split = 0;     // 0: makespan model; else KV splits per prefill tile
+  // prefill tile: a CTA pair on two SMs (M = 256, head_dim 128) or one SM
+  bool use_pair = false;
+  int pair_clusters = 0;  // clusters of two CTAs resident at once (pair kernel)
   int H = 0, Hk = 0, G = 0, D = 0;
   int cap_punits = 0, cap_pgroups = 0, cap_pslots = 0;
   int cap_dunits = 0, cap_dgroups = 0, cap_dslots = 0, cap_dreqs = 0;
@@ -99,7 +111,14 @@ struct pod_attn_ctx {
   PlanLayout lay{};
   // scratch for the planner (reused, sized at create)
   std::vector<PrefillUnit> units_tmp;
-  std::vector<int> units_key;
+  std::vector<int> units_split;
+  std::vector<long long> heap_tmp;
+  std::vector<long long> heap2_tmp;
+  std::vector<long long> parts_len_tmp;
+  std::vector<PrefillUnit> parts_tmp;
+  std::vector<PrefillReq> preq_tmp;
+  std::vector<DecodeReq> dreq_tmp;
+  std::vector<int> dunit_tmp;
 };
 
 namespace {
@@ -110,6 +129,7 @@ PlanLayout plan_layout(const pod_attn_ctx* c) {
   L.ctl = o; o += 64;
   L.ticket = o; o += sizeof(int) * kMaxSmid;
   L.stats = o; o += sizeof(int) * kStatsInts;
+  L.tables0 = o = align_up(o, 64);
   L.pgroup = o; o = align_up(o + sizeof(int) * (size_t)c->cap_pgroups, 64);
   L.dgroup = o; o = align_up(o + sizeof(int) * (size_t)c->cap_dgroups, 64);
   L.tables = o;
@@ -211,61 +231,23 @@ int check_decode(const pod_attn_ctx* c, const pod_decode_args* a) {
 int build_plan(pod_attn_ctx* c, const pod_prefill_args* pa, const pod_decode_args* da,
                bool fused_call, char* h, Plan* P, TmaDescs* T, size_t* copy_bytes) {
   const PlanLayout& L = c->lay;
-  std::memset(h, 0, L.tables);
   const int H = c->H, Hk = c->Hk;
   const int np = (pa ? pa->num_reqs : 0);
   const int nd = (da ? da->num_reqs : 0);
   const bool paged = c->cfg.kv_layout == POD_KV_PAGED;
-  const int slots = c->num_sms * c->slots_per_sm;
+  // persistent prefill workers: CTA pairs, or CTAs of one SM each
+  const int slots = c->use_pair ? c->pair_clusters : c->num_sms * c->slots_per_sm;
 
   // ---- prefill
-  PrefillReq* preq = reinterpret_cast<PrefillReq*>(h + L.preq);
-  PrefillUnit* punits = reinterpret_cast<PrefillUnit*>(h + L.punits);
+  c->preq_tmp.assign(np, PrefillReq{});
+  PrefillReq* preq = c->preq_tmp.data();
   // A unit is two query tiles sharing K/V: a head pair of one KV group at one
   // token tile (G even) or two consecutive token tiles of one head (G odd).
   const bool pair_heads = (c->G % 2) == 0;
-  auto tiles_of = [&](int chunk) -> long long {  // pair units of a chunk, one split each
-    const long long qt = (chunk + kQTile - 1) / kQTile;
-    return pair_heads ? qt * (H / 2) : ((qt + 1) / 2) * H;
-  };
-  long long tiles = 0, w_max = 0;
-  for (int p = 0; p < np; ++p) {
-    if (pa->chunk_lens[p] == 0) continue;
-    tiles += tiles_of(pa->chunk_lens[p]);
-    w_max = std::max<long long>(w_max, (pa->prior_lens[p] + pa->chunk_lens[p] + kKVTile - 1) / kKVTile);
-  }
-  // Splits of the KV range (the same count for every request, clamped per
-  // request below): the s minimising the quantised makespan
-  // ceil(U s / slots) (W / s + o) of U units whose longest has W KV tiles, o
-  // being about two tiles of per-unit overhead (Q load, pipeline fill,
-  // epilogue, merge). Only s with U s <= 2 slots are considered, which also
-  // bounds the partial buffers.
-  int split_base = 1;
-  if (tiles > 0 && c->pre_split > 0) {
-    split_base = c->pre_split;
-    while (split_base > 1 && tiles * split_base > 2LL * slots) --split_base;
-  } else if (tiles > 0 && fused_call && nd > 0) {
-    // One fused launch with decode work: no KV splits. The decode units fill
-    // the SMs an unsplit prefill leaves idle, and the prefill then holds fewer
-    // SMs at once while every other SM streams decode K/V (measured on B200,
-    // llama3_8b: 242 us unsplit against 257 with 2 splits and 265 with 4).
-    split_base = 1;
-  } else if (tiles > 0) {
-    double best = 0.0;
-    for (int sp = 1; sp <= kMaxPrefillSplit && tiles * sp <= 2LL * slots; ++sp) {
-      const double waves = (double)((tiles * sp + slots - 1) / slots);
-      const double cost = waves * ((double)w_max / sp + 2.0);
-      if (sp == 1 || cost < 0.97 * best) {
-        best = cost;
-        split_base = sp;
-      }
-    }
-  }
-  int n_pu = 0, n_pg = 0, n_ps = 0, max_split = 1, q_row = 0;
-  c->units_tmp.clear();
-  c->units_key.clear();
   const int qt_step = pair_heads ? 1 : 2;  // token tiles per unit
   const int h_step = pair_heads ? 2 : 1;   // heads per unit
+  int q_row = 0;
+  c->units_tmp.clear();
   for (int p = 0; p < np; ++p) {
     PrefillReq& R = preq[p];
     const int chunk = pa->chunk_lens[p], prior = pa->prior_lens[p];
@@ -276,50 +258,191 @@ int build_plan(pod_attn_ctx* c, const pod_prefill_args* pa, const pod_decode_arg
     R.kv_len = prior + chunk;
     R.bt_row = p;
     R.pair_heads = pair_heads ? 1 : 0;
+    R.n_split = 1;
     q_row += chunk;
-    if (chunk == 0) {
-      R.n_split = 1;
-      continue;
-    }
-    // KV tiles of the request's first unit (its shortest range); a split keeps
-    // >= 4 tiles of 128 keys
-    const int min_tiles = (prior + std::min(chunk, qt_step * kQTile) + kKVTile - 1) / kKVTile;
-    int split = std::min(split_base, std::max(1, min_tiles / 4));
-    split = std::min(split, kMaxPrefillSplit);
-    R.n_split = split;
-    R.n_kvtiles_max = (prior + chunk + kKVTile - 1) / kKVTile;
-    if (split > 1) {
-      R.group0 = n_pg;
-      R.slot0 = n_ps;
-      n_pg += R.n_qtiles * H;
-      n_ps += R.n_qtiles * H * split;
-    }
-    max_split = std::max(max_split, split);
     for (int qt = 0; qt < R.n_qtiles; qt += qt_step) {
       const int last_qt = std::min(qt + qt_step, R.n_qtiles) - 1;
       const int kv_hi = prior + std::min(chunk, (last_qt + 1) * kQTile);
-      const int work = (kv_hi + kKVTile - 1) / kKVTile / split;
-      for (int hh = 0; hh < H; hh += h_step)
-        for (int sp = 0; sp < split; ++sp) {
-          c->units_tmp.push_back(PrefillUnit{p, hh, qt, sp});
-          c->units_key.push_back(work);
-        }
+      const int work = (kv_hi + kKVTile - 1) / kKVTile;
+      for (int hh = 0; hh < H; hh += h_step) {
+        c->units_tmp.push_back(PrefillUnit{p, hh, qt, 0, 1, 0, 0, work});
+      }
     }
   }
-  n_pu = (int)c->units_tmp.size();
-  if (n_pu > c->cap_punits || n_pg > c->cap_pgroups || n_ps > c->cap_pslots) return POD_ECAPACITY;
-  {
-    // longest units first (LPT) so the tail of the queue is short work
-    std::vector<int> idx(n_pu);
-    for (int i = 0; i < n_pu; ++i) idx[i] = i;
-    std::stable_sort(idx.begin(), idx.end(),
-                     [&](int a, int b) { return c->units_key[a] > c->units_key[b]; });
-    for (int i = 0; i < n_pu; ++i) punits[i] = c->units_tmp[idx[i]];
+  const int n_draft = (int)c->units_tmp.size();
+  // queue order: longest first (LPT), so the tail of the queue is short work;
+  // ties in request, token tile, head and split order
+  auto queue_order = [](const PrefillUnit& a, const PrefillUnit& b) {
+    if (a.work != b.work) return a.work > b.work;
+    if (a.req != b.req) return a.req < b.req;
+    if (a.qtile != b.qtile) return a.qtile < b.qtile;
+    if (a.head != b.head) return a.head < b.head;
+    return a.split < b.split;
+  };
+  std::sort(c->units_tmp.begin(), c->units_tmp.end(), queue_order);
+  // KV splits per unit. A split keeps >= 4 KV tiles. Candidates: the same
+  // count for every unit (the summary's "at most two full waves": units x
+  // splits <= 2 slots), or splitting only the units of the last, partial
+  // wave; each is scored by the finish time of a longest-first assignment of
+  // the parts to the slots (what the persistent queue does), with two tiles
+  // of per-part overhead (query load, pipeline fill, epilogue, merge).
+  std::vector<int>& split = c->units_split;
+  split.assign(n_draft, 1);
+  auto max_split_of = [&](int u) {
+    return std::max(1, std::min(kMaxPrefillSplit, c->units_tmp[u].work / 4));
+  };
+  auto makespan = [&](const std::vector<int>& sp) -> long long {
+    // parts in queue order: by part length, longest first
+    std::vector<long long>& parts = c->heap_tmp;
+    parts.clear();
+    for (int u = 0; u < n_draft; ++u) {
+      const long long w = c->units_tmp[u].work;
+      for (int k = 0; k < sp[u]; ++k)
+        parts.push_back((w * (k + 1)) / sp[u] - (w * k) / sp[u] + 2);
+    }
+    std::sort(parts.begin(), parts.end(), std::greater<long long>());
+    // each part goes to the slot that frees first (a min-heap of finish times)
+    std::vector<long long>& hp = c->heap2_tmp;
+    const size_t n0 = std::min(parts.size(), (size_t)std::max(slots, 1));
+    hp.assign(parts.begin(), parts.begin() + n0);
+    long long end = n0 ? hp.front() : 0;
+    std::make_heap(hp.begin(), hp.end(), std::greater<long long>());
+    for (size_t i = n0; i < parts.size(); ++i) {
+      std::pop_heap(hp.begin(), hp.end(), std::greater<long long>());
+      hp.back() += parts[i];
+      end = std::max(end, hp.back());
+      std::push_heap(hp.begin(), hp.end(), std::greater<long long>());
+    }
+    return end;
+  };
+  auto fits = [&](const std::vector<int>& sp) {
+    long long groups = 0, tiles = 0;
+    for (int u = 0; u < n_draft; ++u)
+      if (sp[u] > 1) {
+        groups += 2;
+        tiles += 2LL * sp[u];
+      }
+    return groups <= c->cap_pgroups && tiles <= c->cap_pslots;
+  };
+  if (n_draft > 0 && c->pre_split > 0) {
+    int s_all = c->pre_split;
+    while (s_all > 1 && (long long)n_draft * s_all > 2LL * slots) --s_all;
+    for (int u = 0; u < n_draft; ++u) split[u] = std::min(s_all, max_split_of(u));
+    if (!fits(split)) split.assign(n_draft, 1);
+  } else if (n_draft > 0) {
+    const long long base = makespan(split);
+    bool consider = true;
+    if (fused_call && nd > 0) {
+      // One fused launch that also carries decodes: split only when the
+      // prefill is the longer phase. Otherwise the decode units fill the
+      // slots an unsplit prefill leaves idle, and the prefill holds fewer SMs
+      // at once while the others stream decode K/V (measured on B200,
+      // Llama-3-8B batch: 242 us unsplit against 257 with 2 splits).
+      const double tile_us = c->use_pair ? 0.75 : (c->D == 128 ? 2.0 : 1.2);
+      double kv_bytes = 0.0;
+      for (int r = 0; r < nd; ++r) kv_bytes += (double)da->ctx_lens[r] * Hk * c->D * 4.0;
+      consider = (double)base * tile_us > kv_bytes / 6.0e6;  // decode at ~6 TB/s
+    }
+    if (consider) {
+      long long best = base;
+      std::vector<int> cand(n_draft);
+      auto try_cand = [&]() {
+        if (!fits(cand)) return;
+        const long long t = makespan(cand);
+        if (t < (best * 97) / 100) {
+          best = t;
+          split = cand;
+        }
+      };
+      for (int s_all = 2; s_all <= kMaxPrefillSplit && (long long)n_draft * s_all <= 2LL * slots;
+           ++s_all) {
+        for (int u = 0; u < n_draft; ++u) cand[u] = std::min(s_all, max_split_of(u));
+        try_cand();
+      }
+      const int tail = n_draft > slots ? n_draft % slots : 0;
+      if (tail > 0) {
+        // The tail units are the shortest, so their parts queue after every
+        // unsplit unit: run the unsplit prefix once, then each tail split.
+        std::vector<long long>& hp0 = c->heap_tmp;
+        hp0.clear();
+        long long end0 = 0;
+        const int prefix = n_draft - tail;
+        for (int u = 0; u < prefix; ++u) {
+          const long long w = c->units_tmp[u].work + 2;
+          if ((int)hp0.size() < slots) {
+            hp0.push_back(w);
+            end0 = std::max(end0, w);
+            if ((int)hp0.size() == slots)
+              std::make_heap(hp0.begin(), hp0.end(), std::greater<long long>());
+            continue;
+          }
+          std::pop_heap(hp0.begin(), hp0.end(), std::greater<long long>());
+          hp0.back() += w;
+          end0 = std::max(end0, hp0.back());
+          std::push_heap(hp0.begin(), hp0.end(), std::greater<long long>());
+        }
+        for (int s_tail = 2; s_tail <= 4; ++s_tail) {
+          for (int u = 0; u < n_draft; ++u)
+            cand[u] = (u >= prefix) ? std::min(s_tail, max_split_of(u)) : 1;
+          if (!fits(cand)) continue;
+          std::vector<long long>& tp = c->parts_len_tmp;
+          tp.clear();
+          for (int u = prefix; u < n_draft; ++u) {
+            const long long w = c->units_tmp[u].work;
+            for (int k = 0; k < cand[u]; ++k)
+              tp.push_back((w * (k + 1)) / cand[u] - (w * k) / cand[u] + 2);
+          }
+          std::sort(tp.begin(), tp.end(), std::greater<long long>());
+          std::vector<long long>& hp = c->heap2_tmp;
+          hp = hp0;  // prefix >= slots: a full heap of finish times
+          long long end = end0;
+          for (long long w : tp) {
+            std::pop_heap(hp.begin(), hp.end(), std::greater<long long>());
+            hp.back() += w;
+            end = std::max(end, hp.back());
+            std::push_heap(hp.begin(), hp.end(), std::greater<long long>());
+          }
+          if (end < (best * 97) / 100) {
+            best = end;
+            split = cand;
+          }
+        }
+      }
+    }
   }
+  // expand the parts; split units get their merge groups and partial slots
+  int n_pg = 0, n_ps = 0, max_split = 1;
+  std::vector<PrefillUnit>& parts = c->parts_tmp;
+  parts.clear();
+  for (int u = 0; u < n_draft; ++u) {
+    PrefillUnit U = c->units_tmp[u];
+    const int sp = split[u];
+    U.n_split = sp;
+    if (sp > 1) {
+      U.group0 = n_pg;
+      U.slot0 = n_ps;
+      n_pg += 2;
+      n_ps += 2 * sp;
+    }
+    max_split = std::max(max_split, sp);
+    preq[U.req].n_split = std::max(preq[U.req].n_split, sp);
+    const int w = U.work;
+    for (int k = 0; k < sp; ++k) {
+      PrefillUnit part = U;
+      part.split = k;
+      part.work = (w * (k + 1)) / sp - (w * k) / sp;
+      parts.push_back(part);
+    }
+  }
+  const int n_pu = (int)parts.size();
+  if (n_pu > c->cap_punits || n_pg > c->cap_pgroups || n_ps > c->cap_pslots) return POD_ECAPACITY;
+  std::sort(parts.begin(), parts.end(), queue_order);
+  const PrefillUnit* punits = parts.data();
 
   // ---- decode
-  DecodeReq* dreq = reinterpret_cast<DecodeReq*>(h + L.dreq);
-  int* dunit = reinterpret_cast<int*>(h + L.dunit);
+  c->dreq_tmp.assign(nd, DecodeReq{});
+  DecodeReq* dreq = c->dreq_tmp.data();
+  std::vector<int>& dunit = c->dunit_tmp;
   // Keys per decode split (a multiple of the 16-key decode tile): the
   // candidate minimising an estimate of the decode makespan on the persistent
   // decode warps. Units are claimed dynamically, so with U units of at most
@@ -361,6 +484,7 @@ int build_plan(pod_attn_ctx* c, const pod_prefill_args* pa, const pod_decode_arg
     }
   }
   int n_du = 0, n_dg = 0, n_ds = 0;
+  dunit.clear();
   for (int r = 0; r < nd; ++r) {
     DecodeReq& R = dreq[r];
     const int len = da->ctx_lens[r];
@@ -378,7 +502,7 @@ int build_plan(pod_attn_ctx* c, const pod_prefill_args* pa, const pod_decode_arg
     }
     const int nu = R.n_split * Hk;
     if (n_du + nu > c->cap_dunits) return POD_ECAPACITY;
-    for (int i = 0; i < nu; ++i) dunit[n_du + i] = r;
+    dunit.insert(dunit.end(), nu, r);
     n_du += nu;
   }
   if (n_dg > c->cap_dgroups || n_ds > c->cap_dslots) return POD_ECAPACITY;
@@ -401,9 +525,9 @@ int build_plan(pod_attn_ctx* c, const pod_prefill_args* pa, const pod_decode_arg
   // finishes in the decode time (all SMs when prefill dominates).
   int p_cap = slots;
   if (c->policy == 5 && n_pu > 0 && nd > 0) {
-    const double tile_us = (c->D == 128 ? 2.0 : 1.2), unit_us = 3.0;
+    const double tile_us = c->use_pair ? 0.75 : (c->D == 128 ? 2.0 : 1.2), unit_us = 3.0;
     double p_sm_us = 0.0;
-    for (int u = 0; u < n_pu; ++u) p_sm_us += c->units_key[u] * tile_us + unit_us;
+    for (int u = 0; u < n_pu; ++u) p_sm_us += punits[u].work * tile_us + unit_us;
     double kv_keys = 0.0;
     for (int r = 0; r < nd; ++r) kv_keys += (double)da->ctx_lens[r];
     const double d_us = kv_keys * Hk * c->D * 4.0 / 6.0e6;  // K and V, bf16, ~6 TB/s
@@ -435,11 +559,25 @@ int build_plan(pod_attn_ctx* c, const pod_prefill_args* pa, const pod_decode_arg
   Q.p_cap = p_cap;
   Q.dec_turn = c->dec_turn;
   Q.wait_budget = kDefaultWaitBudget;
+  // ---- pack the plan: zeroed words, merge counters, then the tables in use
+  const size_t o_pg = L.tables0;
+  const size_t o_dg = align_up(o_pg + sizeof(int) * (size_t)n_pg, 64);
+  const size_t o_preq = align_up(o_dg + sizeof(int) * (size_t)n_dg, 64);
+  const size_t o_pu = align_up(o_preq + sizeof(PrefillReq) * (size_t)np, 64);
+  const size_t o_dreq = align_up(o_pu + sizeof(PrefillUnit) * (size_t)n_pu, 64);
+  const size_t o_du = align_up(o_dreq + sizeof(DecodeReq) * (size_t)nd, 64);
+  const size_t o_end = o_du + sizeof(int) * (size_t)n_du;
+  if (o_end > c->plan_cap) return POD_ECAPACITY;
+  std::memset(h, 0, o_preq);
+  if (np) std::memcpy(h + o_preq, preq, sizeof(PrefillReq) * (size_t)np);
+  if (n_pu) std::memcpy(h + o_pu, punits, sizeof(PrefillUnit) * (size_t)n_pu);
+  if (nd) std::memcpy(h + o_dreq, dreq, sizeof(DecodeReq) * (size_t)nd);
+  if (n_du) std::memcpy(h + o_du, dunit.data(), sizeof(int) * (size_t)n_du);
   char* dp = c->d_plan;
-  Q.preq = reinterpret_cast<const PrefillReq*>(dp + L.preq);
-  Q.punits = reinterpret_cast<const PrefillUnit*>(dp + L.punits);
-  Q.dreq = reinterpret_cast<const DecodeReq*>(dp + L.dreq);
-  Q.dunit_req = reinterpret_cast<const int*>(dp + L.dunit);
+  Q.preq = reinterpret_cast<const PrefillReq*>(dp + o_preq);
+  Q.punits = reinterpret_cast<const PrefillUnit*>(dp + o_pu);
+  Q.dreq = reinterpret_cast<const DecodeReq*>(dp + o_dreq);
+  Q.dunit_req = reinterpret_cast<const int*>(dp + o_du);
   if (np) {
     Q.q_p = static_cast<const uint16_t*>(pa->q);
     Q.o_p = static_cast<uint16_t*>(pa->o);
@@ -465,8 +603,8 @@ int build_plan(pod_attn_ctx* c, const pod_prefill_args* pa, const pod_decode_arg
   Q.ctl = reinterpret_cast<int*>(dp + L.ctl);
   Q.sm_ticket = reinterpret_cast<int*>(dp + L.ticket);
   Q.stats = reinterpret_cast<int*>(dp + L.stats);
-  Q.pgroup_ctr = reinterpret_cast<int*>(dp + L.pgroup);
-  Q.dgroup_ctr = reinterpret_cast<int*>(dp + L.dgroup);
+  Q.pgroup_ctr = reinterpret_cast<int*>(dp + o_pg);
+  Q.dgroup_ctr = reinterpret_cast<int*>(dp + o_dg);
   Q.status = c->d_misc;
   Q.never_set = c->d_misc + 1;
 
@@ -480,7 +618,8 @@ int build_plan(pod_attn_ctx* c, const pod_prefill_args* pa, const pod_decode_arg
       for (int p = 0; p < np; ++p) {
         if (pa->chunk_lens[p] == 0) continue;
         const uint64_t len = (uint64_t)pa->chunk_lens[p] + (uint64_t)pa->prior_lens[p];
-        rc = make_map(c, &T->k[p], pa->k_ptrs[p], (uint64_t)Hk, len, kKVTile);
+        rc = make_map(c, &T->k[p], pa->k_ptrs[p], (uint64_t)Hk, len,
+                      c->use_pair ? kKVTile / 2 : kKVTile);  // the pair loads K in halves
         if (rc) return rc;
         rc = make_map(c, &T->v[p], pa->v_ptrs[p], (uint64_t)Hk, len, kKVTile);
         if (rc) return rc;
@@ -503,19 +642,30 @@ int build_plan(pod_attn_ctx* c, const pod_prefill_args* pa, const pod_decode_arg
   c->last.ratio_num = rho_num;
   c->last.ratio_den = rho_den;
   c->last.prefill_sm_cap = p_cap;
-  size_t used = L.dunit + sizeof(int) * (size_t)n_du;
-  if (n_du == 0) used = L.dreq + sizeof(DecodeReq) * (size_t)nd;
-  if (nd == 0 && n_du == 0) used = L.punits + sizeof(PrefillUnit) * (size_t)n_pu;
-  *copy_bytes = std::max(used, L.tables);
+  c->last.pair_clusters = c->use_pair ? c->pair_clusters : 0;
+  *copy_bytes = o_end;
   c->last.plan_bytes = (long long)*copy_bytes;
   return POD_OK;
 }
 
 int fused_grid(const pod_attn_ctx* c, const Plan& P, bool allow_decode) {
   long long claims = P.n_prefill_units;
+  if (c->use_pair) {  // clusters of two CTAs
+    if (allow_decode) claims += (P.n_decode_units + 2 * kFusedWarps - 1) / (2 * kFusedWarps);
+    const long long g = std::min<long long>(c->pair_clusters, claims);
+    return 2 * (int)std::max<long long>(g, 1);
+  }
   if (allow_decode) claims += (P.n_decode_units + kFusedWarps - 1) / kFusedWarps;
   long long g = std::min<long long>((long long)c->num_sms * c->slots_per_sm, claims);
   return (int)std::max<long long>(g, 1);
+}
+
+// The persistent fused launch (prefill and / or decode units).
+cudaError_t run_fused(const pod_attn_ctx* c, const Plan& P, const TmaDescs& T, bool allow_decode,
+                      cudaStream_t s) {
+  const int grid = fused_grid(c, P, allow_decode);
+  if (c->use_pair) return launch_fused_pair(P, T, grid, 1, allow_decode ? 1 : 0, s);
+  return launch_fused(P, T, grid, 1, allow_decode ? 1 : 0, s);
 }
 
 // Common front half of every call: pick a ring slot, plan, copy the plan.
@@ -625,6 +775,22 @@ int pod_attn_create(pod_attn_ctx** out, const pod_attn_config* cfg) {
     c->pre_split = std::max(0, std::min(kMaxPrefillSplit, std::atoi(e)));
   if (const char* e = std::getenv("POD_ATTN_DEC_SPLIT"))
     c->dec_split = std::max(0, std::atoi(e)) / kDecTile * kDecTile;
+  // The CTA-pair prefill tile (head_dim 128) unless switched off; its
+  // persistent launch uses every cluster of two that fits at once.
+  if (D == 128) {
+    const char* e = std::getenv("POD_ATTN_PREFILL_TILE");
+    if (!(e && !std::strcmp(e, "1sm"))) {
+      int clusters = 0;
+      if (pair_max_clusters(&clusters) != cudaSuccess) return fail(POD_ECUDA);
+      if (clusters >= 1) {
+        c->use_pair = true;
+        c->pair_clusters = clusters;
+        // the pair's prefill tile is fast enough that its units go first:
+        // decode streams beside them on every SM's side warps
+        if (!std::getenv("POD_ATTN_POLICY")) c->policy = 2;
+      }
+    }
+  }
   int dec_blocks = 0;
   if (decode_occupancy(D, &dec_blocks) != cudaSuccess || dec_blocks < 1) return fail(POD_ECUDA);
   c->decode_grid = c->num_sms * dec_blocks;
@@ -665,7 +831,6 @@ int pod_attn_create(pod_attn_ctx** out, const pod_attn_config* cfg) {
     return fail(POD_ECUDA);
   c->encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
   c->units_tmp.reserve(1024);
-  c->units_key.reserve(1024);
   if (cudaDeviceSynchronize() != cudaSuccess) return fail(POD_ECUDA);
   *out = c;
   return POD_OK;
@@ -691,12 +856,11 @@ int pod_attn_hybrid(pod_attn_ctx* c, const pod_prefill_args* pa, const pod_decod
   const bool has_p = P.n_prefill_units > 0, has_d = P.n_decode_units > 0;
   if (!has_p && !has_d) return POD_OK;
   if (mode == POD_MODE_FUSED) {
-    if (launch_fused(P, T, fused_grid(c, P, true), 1, 1, s) != cudaSuccess) return POD_ECUDA;
+    if (run_fused(c, P, T, true, s) != cudaSuccess) return POD_ECUDA;
     return POD_OK;
   }
   if (mode == POD_MODE_SERIAL) {
-    if (has_p && launch_fused(P, T, fused_grid(c, P, false), 1, 0, s) != cudaSuccess)
-      return POD_ECUDA;
+    if (has_p && run_fused(c, P, T, false, s) != cudaSuccess) return POD_ECUDA;
     if (has_d && (launch_decode(P, c->decode_grid, s) != cudaSuccess || launch_merge(P, s) != cudaSuccess))
       return POD_ECUDA;
     return POD_OK;
@@ -704,8 +868,7 @@ int pod_attn_hybrid(pod_attn_ctx* c, const pod_prefill_args* pa, const pod_decod
   // TWO_STREAM
   if (cudaEventRecord(c->ev_fork, s) != cudaSuccess) return POD_ECUDA;
   if (cudaStreamWaitEvent(c->side, c->ev_fork, 0) != cudaSuccess) return POD_ECUDA;
-  if (has_p && launch_fused(P, T, fused_grid(c, P, false), 1, 0, s) != cudaSuccess)
-    return POD_ECUDA;
+  if (has_p && run_fused(c, P, T, false, s) != cudaSuccess) return POD_ECUDA;
   if (has_d && (launch_decode(P, c->decode_grid, c->side) != cudaSuccess || launch_merge(P, c->side) != cudaSuccess))
     return POD_ECUDA;
   if (cudaEventRecord(c->ev_join, c->side) != cudaSuccess) return POD_ECUDA;
@@ -726,7 +889,7 @@ int pod_attn_prefill_only(pod_attn_ctx* c, const pod_prefill_args* pa, void* str
   rc = stage_plan(c, pa, nullptr, false, s, &P, &T);
   if (rc) return rc;
   if (P.n_prefill_units == 0) return POD_OK;
-  return launch_fused(P, T, fused_grid(c, P, false), 1, 0, s) == cudaSuccess ? POD_OK : POD_ECUDA;
+  return run_fused(c, P, T, false, s) == cudaSuccess ? POD_OK : POD_ECUDA;
 }
 
 int pod_attn_decode_only(pod_attn_ctx* c, const pod_decode_args* da, void* stream) {

@@ -615,8 +615,10 @@ __global__ void __launch_bounds__(kFusedThreads, kFusedSlotsPerSm)
             break;
         }
       }
+      // The loop ends only through the role thread 0 posts (0 once the CTA
+      // has aborted): the abort flag can change at any moment (side warps, the
+      // peer CTA), so testing it here could split the warps at bar.sync 1.
       role_sync();
-      if (*abort_flag) break;
     }
   } else if (allow_decode) {
     const int sw = warp - kRoleWarps;
@@ -646,6 +648,228 @@ __global__ void __launch_bounds__(kFusedThreads, kFusedSlotsPerSm)
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ============================================================= CTA-pair fused kernel
+#include "pod_prefill2.cuh"
+
+// One persistent cluster of two 12-warp CTAs per SM pair. The leader CTA's
+// thread 0 takes the tickets (from its SM's counter) and claims prefill units
+// for the pair; it posts each decision to the peer through a mailbox in the
+// peer's shared memory (a remote store plus a remote barrier arrival) and
+// waits for the peer's acknowledgement before posting the next one. A prefill
+// unit runs on both CTAs (pair_*); a decode turn runs on each CTA's role warps
+// independently. Warps 10-11 of both CTAs stream decode units throughout.
+template <int D>
+__global__ void __launch_bounds__(kFusedThreads, 1)
+    pod_fused_pair_kernel(const __grid_constant__ Plan P, const __grid_constant__ TmaDescs T,
+                          int allow_prefill, int allow_decode) {
+  using L = PairLayout<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* sm = smem_raw;
+  const int tid = threadIdx.x;
+  // Both CTAs of the pair have the same layout, so both take this branch or
+  // neither does.
+  if (smem_u32(sm) & 1023u) {  // 128-byte swizzle atoms need 1024-byte alignment
+    if (tid == 0) set_status(P, kStatusUnsupported);
+    return;
+  }
+  const int warp = tid >> 5, lane = tid & 31;
+  const int rank = (int)cluster_ctarank();
+  const uint32_t bars = smem_u32(sm) + L::BAR_OFF;
+  int* misc = reinterpret_cast<int*>(sm + L::MISC_OFF);
+  const uint32_t peer = (uint32_t)(rank ^ 1);
+  const PairAbort pa{reinterpret_cast<volatile int*>(misc + kMiscAbort),
+                     mapa_shared(smem_u32(misc + kMiscAbort), peer)};
+  volatile int* abort_flag = pa.flag;
+
+  if (tid == 0) {
+    for (int i = 0; i < L::N_BARS; ++i) {
+      uint32_t cnt = 1;
+      if (i == L::B_SE || i == L::B_SE + 1 || i == L::B_PF || i == L::B_PF + 1)
+        cnt = 2 * kSoftmaxWarps;  // every softmax warp of both CTAs
+      mbar_init(bars + i * 8, cnt);
+    }
+    fence_mbar_init();
+    for (int i = 0; i < 16; ++i) misc[i] = 0;
+    misc[kMiscPEmpty] = allow_prefill ? 0 : 1;
+    misc[kMiscDEmpty] = allow_decode ? 0 : 1;
+  }
+  // barrier initialisation visible to the peer before any remote arrival
+  cluster_sync_all();
+  if (warp == 0) {
+    tmem_alloc_pair(smem_u32(misc + kMiscTmem), kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = static_cast<uint32_t>(misc[kMiscTmem]);
+
+  // Test hook: one thread waits on a flag nothing sets, with a short budget,
+  // then records the timeout and carries on.
+  if ((P.flags & 0x2) && blockIdx.x == 0 && tid == 0) {
+    const long long t0 = clock64();
+    while (*reinterpret_cast<volatile const int*>(P.never_set) == 0) {
+      if (clock64() - t0 > 2000000LL) {
+        set_status(P, kStatusTimeout);
+        break;
+      }
+    }
+  }
+
+  const uint32_t my_sm = smid() & (kMaxSmid - 1);
+  PairPipe ps = {0u, 0u, 0u, 0u, 0u};
+  uint32_t dec_ring = 0;
+  uint32_t last_commit_bar = 0, last_commit_par = 0;
+  bool issued_mma = false;
+  const uint32_t peer_misc = mapa_shared(smem_u32(misc), peer);
+  const uint32_t peer_bars = mapa_shared(bars, peer);
+
+  auto role_sync = [] { asm volatile("bar.sync 1, %0;" ::"n"(kRoleWarps * 32) : "memory"); };
+  if (warp < kRoleWarps) {
+    uint32_t posts = 0;  // mailbox posts sent (leader) or read (peer)
+    while (true) {
+      if (tid == 0) {
+        int role = 0, unit = -1;
+        if (rank == 0) {
+          if (!*abort_flag) {
+            const int t = atomicAdd(P.sm_ticket + ((P.flags & kFlagGlobalTicket) ? 0 : my_sm), 1);
+            const long long num = P.rho_num, den = P.rho_den > 0 ? P.rho_den : 1;
+            bool want_p = ((long long)(t + 1) * num) / den > ((long long)t * num) / den;
+            if ((P.flags & kFlagFrontPolicy) && t < kFusedSlotsPerSm) want_p = true;
+            if (P.flags & kFlagBalancedPolicy) want_p = (int)(blockIdx.x >> 1) < P.p_cap;
+            for (int attempt = 0; attempt < 2 && role == 0; ++attempt, want_p = !want_p) {
+              if (want_p && !misc[kMiscPEmpty]) {
+                const int u = atomicAdd(P.ctl + 0, 1);
+                if (u < P.n_prefill_units) {
+                  role = 1;
+                  unit = u;
+                } else {
+                  misc[kMiscPEmpty] = 1;
+                }
+              } else if (!want_p && !misc[kMiscDEmpty]) {
+                role = 2;
+                unit = 0;
+              }
+            }
+            if (role && (P.flags & 0x1)) atomicAdd(P.stats + my_sm * 2 + (role - 1), 1);
+          }
+          // the peer must have read the previous post before it is overwritten
+          if (posts > 0 && !pwait_c(bars + L::B_ACK * 8, (posts - 1) & 1, P, pa)) role = 0;
+          st_cluster_u32(peer_misc + 4 * kMiscPending, 1u);
+          st_cluster_u32(peer_misc + 4 * kMiscMbRole, (uint32_t)role);
+          st_cluster_u32(peer_misc + 4 * kMiscMbUnit, (uint32_t)unit);
+          mbar_arrive_cluster(peer_bars + L::B_MB * 8);
+        } else {
+          if (pwait_c(bars + L::B_MB * 8, posts & 1, P, pa)) {
+            role = *reinterpret_cast<volatile int*>(misc + kMiscMbRole);
+            unit = *reinterpret_cast<volatile int*>(misc + kMiscMbUnit);
+            *reinterpret_cast<volatile int*>(misc + kMiscPending) = 0;
+            mbar_arrive_cluster(mapa_shared(bars + L::B_ACK * 8, 0));
+          }
+        }
+        ++posts;
+        misc[kMiscRole] = role;
+        misc[kMiscUnit] = unit;
+      }
+      role_sync();
+      const int role = misc[kMiscRole];
+      const int unit = misc[kMiscUnit];
+      if (role == 0) break;
+      if (role == 1) {
+        const PrefillRange pr = prefill_range(P, unit);
+        if (warp < kSoftmaxWarps) {
+          pair_softmax<D>(P, pr, rank, sm, tmem, ps, tid, pa, misc + kMiscMerge);
+        } else if (warp == kSoftmaxWarps) {
+          if (lane == 0 && rank == 0) {
+            issued_mma = true;
+            pair_mma<D>(P, pr, sm, tmem, ps, last_commit_bar, last_commit_par, pa);
+          }
+          __syncwarp();
+        } else if (warp == kSoftmaxWarps + 1) {
+          if (lane == 0) pair_producer<D>(P, T, pr, rank, sm, ps, pa);
+          __syncwarp();
+        }
+      } else {
+        // decode turn: each role warp claims up to dec_turn units; once every
+        // prefill unit has been claimed it keeps claiming until the decode
+        // queue is empty. The peer also ends its turn when the leader has
+        // posted a new decision (the pair is wanted for a prefill unit).
+        for (int k = 0;; ++k) {
+          if (k >= P.dec_turn && !(P.flags & kFlagBalancedPolicy) &&
+              *reinterpret_cast<volatile const int*>(P.ctl + 0) < P.n_prefill_units)
+            break;
+          if (rank == 1 && *reinterpret_cast<volatile int*>(misc + kMiscPending)) break;
+          int u = 0;
+          if (lane == 0) u = atomicAdd(P.ctl + 1, 1);
+          u = __shfl_sync(0xffffffffu, u, 0);
+          if (u >= P.n_decode_units) {
+            if (lane == 0) misc[kMiscDEmpty] = 1;
+            break;
+          }
+          if (!decode_unit_warp<D, L::ROLE_DEC_ST>(P, u, sm + warp * L::ROLE_DEC_WARP,
+                                                  bars + (L::B_DEC + warp * L::ROLE_DEC_ST) * 8,
+                                                  dec_ring, lane, true, abort_flag))
+            break;
+        }
+      }
+      // The loop ends only through the role thread 0 posts (0 once the CTA
+      // has aborted): the abort flag can change at any moment (side warps, the
+      // peer CTA), so testing it here could split the warps at bar.sync 1.
+      role_sync();
+    }
+  } else if (allow_decode) {
+    const int sw = warp - kRoleWarps;
+    uint32_t side_ring = 0;
+    while (!*abort_flag) {
+      int u = 0;
+      if (lane == 0) u = atomicAdd(P.ctl + 1, 1);
+      u = __shfl_sync(0xffffffffu, u, 0);
+      if (u >= P.n_decode_units) {
+        if (lane == 0) misc[kMiscDEmpty] = 1;
+        break;
+      }
+      if (!decode_unit_warp<D, L::SIDE_DEC_ST>(
+              P, u, sm + L::SIDE_OFF + sw * L::SIDE_DEC_WARP,
+              bars + (L::B_DEC + kRoleWarps * L::ROLE_DEC_ST + sw * L::SIDE_DEC_ST) * 8, side_ring,
+              lane, true, abort_flag))
+        break;
+    }
+  }
+  // Teardown. After an abort, wait (bounded) for this CTA's own async work:
+  // the MMAs the leader issued, and the loads the producers issued (a peer's
+  // loads complete on the leader's barriers, so the peer gives them a short
+  // grace period).
+  if (*abort_flag) {
+    if (warp == kSoftmaxWarps && lane == 0 && issued_mma && last_commit_bar)
+      drain_bar(last_commit_bar, last_commit_par, P.wait_budget);
+    if (warp == kSoftmaxWarps + 1 && lane == 0) {
+      if (rank == 0) {
+        if (ps.q > 0) drain_bar(bars + L::B_QF * 8, (ps.q - 1) & 1, P.wait_budget);
+        for (uint32_t k = 0; k < (uint32_t)L::KS && k < ps.kissued; ++k) {
+          const uint32_t it = ps.kissued - 1 - k;
+          drain_bar(bars + (L::B_KF + it % L::KS) * 8, (it / L::KS) & 1, P.wait_budget);
+        }
+        for (uint32_t k = 0; k < (uint32_t)L::VS && k < ps.vissued; ++k) {
+          const uint32_t it = ps.vissued - 1 - k;
+          drain_bar(bars + (L::B_VF + it % L::VS) * 8, (it / L::VS) & 1, P.wait_budget);
+        }
+      } else {
+        const long long t0 = clock64();
+        while (clock64() - t0 < 4000000LL) {
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  // neither CTA leaves (or frees TMEM) while the other may still touch its
+  // shared memory or the pair's tensor memory
+  cluster_sync_all();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, kTmemCols);
   }
 }
 
@@ -713,7 +937,47 @@ static cudaError_t set_attrs() {
                               DecodeLayout<D>::SMEM_BYTES);
 }
 
-cudaError_t kernels_init(int D) { return D == 128 ? set_attrs<128>() : set_attrs<64>(); }
+cudaError_t kernels_init(int D) {
+  if (D == 128) {
+    cudaError_t e = set_attrs<128>();
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(pod_fused_pair_kernel<128>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                PairLayout<128>::SMEM_BYTES);
+  }
+  return set_attrs<64>();
+}
+
+static cudaLaunchConfig_t pair_config(int grid, cudaStream_t s, cudaLaunchAttribute* attr) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid, 1, 1);
+  cfg.blockDim = dim3(kFusedThreads, 1, 1);
+  cfg.dynamicSmemBytes = PairLayout<128>::SMEM_BYTES;
+  cfg.stream = s;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cfg;
+}
+
+// Clusters of two pair CTAs that fit on the device at once (0: none).
+cudaError_t pair_max_clusters(int* clusters) {
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = pair_config(2, nullptr, attr);
+  return cudaOccupancyMaxActiveClusters(clusters, pod_fused_pair_kernel<128>, &cfg);
+}
+
+// grid = 2 x clusters (head_dim 128 only).
+cudaError_t launch_fused_pair(const Plan& P, const TmaDescs& T, int grid, int allow_prefill,
+                              int allow_decode, cudaStream_t s) {
+  if (P.D != 128 || grid < 2 || (grid & 1)) return cudaErrorInvalidValue;
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = pair_config(grid, s, attr);
+  return cudaLaunchKernelEx(&cfg, pod_fused_pair_kernel<128>, P, T, allow_prefill, allow_decode);
+}
 
 int fused_smem_bytes(int D) {
   return D == 128 ? FusedLayout<128>::SMEM_BYTES : FusedLayout<64>::SMEM_BYTES;

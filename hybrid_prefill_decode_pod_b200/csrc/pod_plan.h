@@ -33,7 +33,7 @@ constexpr int kFusedDecStages = 2;    // per-warp decode ring depth in the fused
 constexpr int kDecodeWarps = 6;       // warps (virtual decode units) per decode-only CTA
 constexpr int kDecodeStages = 2;      // per-warp ring depth in the decode-only kernel
 constexpr int kMaxGroup = 8;          // query heads per KV head (mma N = 8)
-constexpr int kTmemCols = 512;        // TMEM columns per CTA: O0, O1, S0, S1 (128 each)
+constexpr int kTmemCols = 512;        // TMEM columns per CTA (all of an SM's tensor memory)
 constexpr int kMaxSmid = 256;         // per-SM ticket slots (indexed by %smid)
 constexpr long long kDefaultWaitBudget = 2000000000LL;  // cycles (~1 s at 2 GHz)
 // Plan::flags bits set by the library itself (the low byte carries the
@@ -45,15 +45,18 @@ constexpr int kFlagPoisonOnStatus = 0x800;  // merge writes NaN when the status 
 
 struct PrefillReq {
   int prior, chunk, q_row0, n_qtiles;
-  int kv_len, bt_row, n_split, group0;  // group0: first merge group of this request
-  int slot0, n_kvtiles_max, pair_heads, pad1;  // slot0: first partial slot (split
-                                               // requests); pair_heads: see PrefillUnit
+  int kv_len, bt_row, n_split, pair_heads;  // n_split: largest split count of its units;
+                                            // pair_heads: see PrefillUnit
 };
 
 // Two query tiles: heads (head, head + 1) at token tile qtile when the
 // request's pair_heads is set, else token tiles (qtile, qtile + 1) of head.
+// The unit covers KV split `split` of `n_split` of the pair's key range. A
+// split pair (n_split > 1) owns merge groups group0 (tile 0) and group0 + 1
+// (tile 1) and partial slots slot0 + i * n_split + s for tile i, split s.
 struct PrefillUnit {
   int req, head, qtile, split;
+  int n_split, group0, slot0, work;  // work: KV tiles of this split (planner's sort key)
 };
 
 struct DecodeReq {

@@ -22,10 +22,12 @@
 // Included by pod_kernels.cu inside namespace pod, after the decode code.
 
 struct PrefillRange {
-  int req, split;
+  int req, split, n_split;
   int head[2], qtile[2];  // the unit's two query tiles
   int valid1;             // tile 1 exists (a token-tile pair may run past the chunk)
   int t0, n;              // first KV tile and number of KV tiles
+  int group[2];           // merge group of each tile (split units)
+  int slot_base[2];       // first partial slot of each tile (split units)
 };
 
 POD_DEV PrefillRange prefill_range(const Plan& P, int u) {
@@ -34,6 +36,11 @@ POD_DEV PrefillRange prefill_range(const Plan& P, int u) {
   PrefillRange pr;
   pr.req = U.req;
   pr.split = U.split;
+  pr.n_split = U.n_split;
+  pr.group[0] = U.group0;
+  pr.group[1] = U.group0 + 1;
+  pr.slot_base[0] = U.slot0;
+  pr.slot_base[1] = U.slot0 + U.n_split;
   if (R.pair_heads) {
     pr.head[0] = U.head;
     pr.head[1] = U.head + 1;
@@ -48,8 +55,8 @@ POD_DEV PrefillRange prefill_range(const Plan& P, int u) {
   const int last_qt = pr.valid1 ? pr.qtile[1] : pr.qtile[0];
   const int kv_hi = R.prior + min(R.chunk, (last_qt + 1) * kQTile);
   const int n_all = (kv_hi + kKVTile - 1) / kKVTile;
-  pr.t0 = (int)((long long)U.split * n_all / R.n_split);
-  pr.n = (int)((long long)(U.split + 1) * n_all / R.n_split) - pr.t0;
+  pr.t0 = (int)((long long)U.split * n_all / U.n_split);
+  pr.n = (int)((long long)(U.split + 1) * n_all / U.n_split) - pr.t0;
   return pr;
 }
 
@@ -364,7 +371,7 @@ POD_DEV bool prefill_softmax(const Plan& P, const PrefillRange& pr, uint8_t* sm,
   const size_t out_row = (size_t)(R.q_row0 + q_local);
   const float lse2 = (l_run > 0.f) ? (m_run + log2f(l_run)) : -INFINITY;
   const int bar_id = 2 + i;  // named barrier of this warp group (128 threads)
-  if (R.n_split <= 1) {
+  if (pr.n_split <= 1) {
     if (failed) return false;
     const float inv = 1.f / l_run;
 #pragma unroll
@@ -390,8 +397,7 @@ POD_DEV bool prefill_softmax(const Plan& P, const PrefillRange& pr, uint8_t* sm,
   // Split partial of this tile: O normalised by its own sum (fp32) and the
   // natural-log LSE of its KV range. O is stored [slot][d / 4][row] in float4
   // units, so the 32 rows of a warp touch 512 contiguous bytes per access.
-  const int gidx = qtile * P.H + head;
-  const int slot0 = R.slot0 + gidx * R.n_split;
+  const int slot0 = pr.slot_base[i];
   const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
   float4* part = reinterpret_cast<float4*>(P.ppart_o);
   {
@@ -414,8 +420,8 @@ POD_DEV bool prefill_softmax(const Plan& P, const PrefillRange& pr, uint8_t* sm,
   asm volatile("bar.sync %0, 128;" ::"r"(bar_id) : "memory");
   if ((tid & 127) == 0) {
     // a missing tile has no group; after a failure nobody merges
-    const int old = (*abort_flag || !tile_ok) ? -1 : atomicAdd(P.pgroup_ctr + R.group0 + gidx, 1);
-    s_flag[i] = (old == R.n_split - 1);
+    const int old = (*abort_flag || !tile_ok) ? -1 : atomicAdd(P.pgroup_ctr + pr.group[i], 1);
+    s_flag[i] = (old == pr.n_split - 1);
   }
   asm volatile("bar.sync %0, 128;" ::"r"(bar_id) : "memory");
   if (s_flag[i] && !failed && valid) {
@@ -423,7 +429,7 @@ POD_DEV bool prefill_softmax(const Plan& P, const PrefillRange& pr, uint8_t* sm,
     // always in split order so the result does not depend on which split
     // finished last: O = sum_s w_s O_s / sum_s w_s, w_s = exp(LSE_s - max LSE).
     __threadfence();
-    const int ns = R.n_split;
+    const int ns = pr.n_split;
     const float* pl = P.ppart_lse + (size_t)slot0 * kQTile + row;
     float m = -INFINITY;
     for (int sp = 0; sp < ns; ++sp) m = fmaxf(m, __ldcg(pl + (size_t)sp * kQTile));

@@ -85,7 +85,7 @@ class PlanInfo(ctypes.Structure):
                 ("decode_units", ctypes.c_int), ("decode_split_len", ctypes.c_int),
                 ("ratio_num", ctypes.c_int), ("ratio_den", ctypes.c_int),
                 ("plan_bytes", ctypes.c_longlong), ("prefill_sm_cap", ctypes.c_int),
-                ("reserved", ctypes.c_int)]
+                ("pair_clusters", ctypes.c_int)]
 
     def as_dict(self):
         return {k: getattr(self, k) for k, _ in self._fields_}

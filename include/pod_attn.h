@@ -167,7 +167,8 @@ typedef struct {
   int ratio_num, ratio_den;  /* prefill share of claims per SM               */
   long long plan_bytes;      /* bytes copied host -> device for the plan      */
   int prefill_sm_cap;        /* fused CTAs that take prefill work first       */
-  int reserved;
+  int pair_clusters;         /* prefill on CTA pairs: clusters of two CTAs;
+                                0 when each prefill unit runs on one SM       */
 } pod_plan_info;
 
 /* Per-SM role counts gathered with POD_FLAG_STATS (the "virtual CTA mix"). */

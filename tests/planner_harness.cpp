@@ -8,7 +8,8 @@
 //
 // Usage: planner_harness H Hk D sms decode_grid policy fused pre_split dec_split
 //                        paged "prior:chunk,..." "len,..." max_prefill_tokens
-//                        max_decode_reqs max_kv_tokens
+//                        max_decode_reqs max_kv_tokens pair_clusters
+// (pair_clusters 0: prefill units on one SM each; else on that many CTA pairs)
 #include "pod_attn_api.cpp"
 
 #include <cstdio>
@@ -24,9 +25,14 @@ cudaError_t launch_fused(const Plan&, const TmaDescs&, int, int, int, cudaStream
 cudaError_t launch_decode(const Plan&, int, cudaStream_t) { std::abort(); }
 cudaError_t decode_occupancy(int, int*) { return cudaErrorNotSupported; }
 cudaError_t launch_merge(const Plan&, cudaStream_t) { std::abort(); }
+cudaError_t pair_max_clusters(int*) { return cudaErrorNotSupported; }
+cudaError_t launch_fused_pair(const Plan&, const TmaDescs&, int, int, int, cudaStream_t) {
+  std::abort();
+}
 }  // namespace pod
 
 static int g_maps = 0;
+static std::vector<int> g_boxes;  // rows per box of each map, in encoding order
 static CUresult fake_encode(CUtensorMap*, CUtensorMapDataType dt, cuuint32_t rank, void* base,
                             const cuuint64_t* dims, const cuuint64_t* strides,
                             const cuuint32_t* box, const cuuint32_t*, CUtensorMapInterleave,
@@ -39,6 +45,8 @@ static CUresult fake_encode(CUtensorMap*, CUtensorMapDataType dt, cuuint32_t ran
   if ((reinterpret_cast<uintptr_t>(base) & 15u) || (strides[0] & 15u) || (strides[1] & 15u))
     return CUDA_ERROR_INVALID_VALUE;
   if (box[0] != 64 || box[1] != 1 || dims[0] % 64) return CUDA_ERROR_INVALID_VALUE;
+  if (box[2] != 16 && box[2] != 64 && box[2] != 128) return CUDA_ERROR_INVALID_VALUE;
+  g_boxes.push_back((int)box[2]);
   return CUDA_SUCCESS;
 }
 
@@ -55,8 +63,8 @@ static std::vector<long long> parse_list(const std::string& s) {
 }
 
 int main(int argc, char** argv) {
-  if (argc != 16) {
-    std::fprintf(stderr, "expected 15 arguments\n");
+  if (argc != 17) {
+    std::fprintf(stderr, "expected 16 arguments\n");
     return 2;
   }
   pod_attn_ctx c;
@@ -82,10 +90,11 @@ int main(int argc, char** argv) {
   c.cfg.max_prefill_reqs = kMaxPrefillReqs;
   c.cfg.max_decode_reqs = std::atoi(argv[14]);
   c.cfg.max_kv_tokens = std::atoll(argv[15]);
+  c.pair_clusters = std::atoi(argv[16]);
+  c.use_pair = c.pair_clusters > 0;
   c.encode = fake_encode;
   size_context(&c);
   c.units_tmp.reserve(1024);
-  c.units_key.reserve(1024);
   std::vector<char> h(c.plan_cap + 64), dplan(c.plan_cap + 64);
   c.d_plan = dplan.data();  // only a base address here: the planner never dereferences it
 
@@ -144,13 +153,31 @@ int main(int argc, char** argv) {
 
   std::printf("{\"status\": %d", rc);
   if (rc == POD_OK) {
-    const PlanLayout& L = c.lay;
-    const PrefillReq* preq = reinterpret_cast<const PrefillReq*>(h.data() + L.preq);
-    const PrefillUnit* pu = reinterpret_cast<const PrefillUnit*>(h.data() + L.punits);
-    const DecodeReq* dreq = reinterpret_cast<const DecodeReq*>(h.data() + L.dreq);
-    const int* du = reinterpret_cast<const int*>(h.data() + L.dunit);
+    // the plan's device pointers are offsets from the stand-in buffer base,
+    // and the host slot has the same layout
+    auto at = [&](const void* dev) { return h.data() + ((const char*)dev - c.d_plan); };
+    const PrefillReq* preq = reinterpret_cast<const PrefillReq*>(at(P.preq));
+    const PrefillUnit* pu = reinterpret_cast<const PrefillUnit*>(at(P.punits));
+    const DecodeReq* dreq = reinterpret_cast<const DecodeReq*>(at(P.dreq));
+    const int* du = reinterpret_cast<const int*>(at(P.dunit_req));
+    // every table lies inside the bytes the call copies, and the zeroed words
+    // (queue heads, tickets, merge counters) are zero
+    const size_t ends[4] = {(size_t)((const char*)(P.preq + np) - c.d_plan),
+                            (size_t)((const char*)(P.punits + P.n_prefill_units) - c.d_plan),
+                            (size_t)((const char*)(P.dreq + nd) - c.d_plan),
+                            (size_t)((const char*)(P.dunit_req + P.n_decode_units) - c.d_plan)};
+    bool inside = true;
+    for (size_t e : ends) inside = inside && e <= bytes && e <= c.plan_cap;
+    bool zeroed = true;
+    for (size_t i = 0; i < (size_t)((const char*)P.preq - c.d_plan); ++i) zeroed = zeroed && !h[i];
+    std::printf(", \"tables_inside_copy\": %s, \"counters_zeroed\": %s", inside ? "true" : "false",
+                zeroed ? "true" : "false");
     std::printf(", \"slots\": %d, \"flags\": %d, \"p_cap\": %d, \"rho\": [%d, %d]",
-                c.num_sms * c.slots_per_sm, P.flags, P.p_cap, P.rho_num, P.rho_den);
+                c.use_pair ? c.pair_clusters : c.num_sms * c.slots_per_sm, P.flags, P.p_cap,
+                P.rho_num, P.rho_den);
+    std::printf(", \"boxes\": [");
+    for (size_t i = 0; i < g_boxes.size(); ++i) std::printf("%s%d", i ? ", " : "", g_boxes[i]);
+    std::printf("]");
     std::printf(", \"plan_bytes\": %zu, \"maps\": %d, \"dec_split_len\": %d", bytes, g_maps,
                 P.dec_split_len);
     std::printf(", \"caps\": {\"punits\": %d, \"pgroups\": %d, \"pslots\": %d, \"dunits\": %d}",
@@ -158,15 +185,14 @@ int main(int argc, char** argv) {
     std::printf(", \"preq\": [");
     for (int i = 0; i < np; ++i)
       std::printf("%s{\"prior\": %d, \"chunk\": %d, \"q_row0\": %d, \"n_qtiles\": %d, "
-                  "\"kv_len\": %d, \"n_split\": %d, \"group0\": %d, \"slot0\": %d, "
-                  "\"pair_heads\": %d}",
+                  "\"kv_len\": %d, \"n_split\": %d, \"pair_heads\": %d}",
                   i ? ", " : "", preq[i].prior, preq[i].chunk, preq[i].q_row0, preq[i].n_qtiles,
-                  preq[i].kv_len, preq[i].n_split, preq[i].group0, preq[i].slot0,
-                  preq[i].pair_heads);
+                  preq[i].kv_len, preq[i].n_split, preq[i].pair_heads);
     std::printf("], \"punits\": [");
     for (int u = 0; u < P.n_prefill_units; ++u)
-      std::printf("%s[%d, %d, %d, %d]", u ? ", " : "", pu[u].req, pu[u].head, pu[u].qtile,
-                  pu[u].split);
+      std::printf("%s[%d, %d, %d, %d, %d, %d, %d, %d]", u ? ", " : "", pu[u].req, pu[u].head,
+                  pu[u].qtile, pu[u].split, pu[u].n_split, pu[u].group0, pu[u].slot0,
+                  pu[u].work);
     std::printf("], \"dreq\": [");
     for (int i = 0; i < nd; ++i)
       std::printf("%s{\"len\": %d, \"n_split\": %d, \"unit0\": %d, \"group0\": %d, \"slot0\": %d}",

@@ -66,23 +66,47 @@ def test_paged_matches_contiguous_bitwise_and_oracle():
     assert bitwise_equal(paged, contig)
 
 
-def test_run_to_run_bitwise_and_modes_bitwise():
+@pytest.mark.parametrize("tile", ["pair", "1sm"])
+def test_run_to_run_bitwise_and_modes_bitwise(tile):
     b = W.make_custom(8, 2, 128, [(2000, 300)], [100, 5000, 7000, 64], seed=13)
-    a1, p1 = run(b, "fused")
-    a2, _ = run(b, "fused")
+    with plan_env(POD_ATTN_PREFILL_TILE=tile):
+        a1, p1 = run(b, "fused")
+        a2, _ = run(b, "fused")
     assert bitwise_equal(a1, a2)
-    # FUSED leaves the prefill unsplit when decodes share the launch, the
-    # separate-launch modes may split it; on the same plan all three modes
-    # give identical bits
+    assert (p1["pair_clusters"] > 0) == (tile == "pair")
+    # FUSED may plan the prefill split differently from the separate-launch
+    # modes (it leaves it unsplit when decode is the longer phase); on the
+    # same plan all three modes give identical bits
     for split in ("1", "3"):
-        with plan_env(POD_ATTN_PREFILL_SPLIT=split):
+        with plan_env(POD_ATTN_PREFILL_SPLIT=split, POD_ATTN_PREFILL_TILE=tile):
             f, pf = run(b, "fused")
             s1, ps = run(b, "serial")
             t1, _ = run(b, "two_stream")
         assert pf["prefill_split"] == ps["prefill_split"] == int(split)
         assert bitwise_equal(f, s1)
         assert bitwise_equal(f, t1)
-    assert p1["prefill_split"] == 1
+
+
+PAIR_SHAPES = [
+    # the one-SM prefill tile against the CTA-pair tile, both against the oracle
+    (8, 2, 128, [(300, 200)], [1, 17, 1000]),
+    (6, 2, 128, [(900, 300)], [50, 700]),                         # G = 3: token-tile pairs
+    (4, 4, 128, [(1000, 64)], [2048]),                            # G = 1, missing 2nd tile
+    (16, 2, 128, [(0, 130), (77, 257)], [5, 4096]),               # G = 8, two requests
+]
+
+
+@pytest.mark.parametrize("shape", PAIR_SHAPES)
+def test_pair_and_one_sm_prefill_tiles_match_oracle(shape):
+    H, Hk, d, pre, ctx = shape
+    b = W.make_custom(H, Hk, d, pre, ctx, seed=7)
+    ref = oracle.hybrid(b)
+    for tile in ("pair", "1sm"):
+        for split in ("0", "3"):
+            with plan_env(POD_ATTN_PREFILL_TILE=tile, POD_ATTN_PREFILL_SPLIT=split):
+                out, plan = run(b, "fused")
+            assert (plan["pair_clusters"] > 0) == (tile == "pair")
+            compare(ref, out)
 
 
 def test_prefill_only_and_decode_only_match_hybrid():
