@@ -481,6 +481,87 @@ def run_gpu(args, rank, world, local):
     return 0
 
 
+# Variants of the chunked-prompt study (the POD-Attention summary, §4.2.3 and
+# §5.4.3 / Table 8: limiting the prefill's KV splits to two waves; §4.2.2 /
+# §5.4.1: the prefill tile's size). Each is a set of planner levers read when
+# a context is created.
+SWEEP_VARIANTS = {
+    "pair_model": {},                                        # CTA-pair tile, split model
+    "pair_nosplit": {"POD_ATTN_PREFILL_SPLIT": "1"},
+    "pair_uncapped8": {"POD_ATTN_PREFILL_SPLIT": "-8"},      # 8 splits, two-wave cap off
+    "1sm_model": {"POD_ATTN_PREFILL_TILE": "1sm"},           # one-SM pair tile, split model
+    "1sm_uncapped8": {"POD_ATTN_PREFILL_TILE": "1sm", "POD_ATTN_PREFILL_SPLIT": "-8"},
+}
+SWEEP_POLICIES = {  # the fused kernel's role policy (§4.1, §5.4.2 / Figure 14)
+    "prefill_first": {"POD_ATTN_POLICY": "prefill_first"},
+    "front": {"POD_ATTN_POLICY": "front"},
+    "even": {"POD_ATTN_POLICY": "even"},
+    "proportional": {"POD_ATTN_POLICY": "proportional"},
+    "balanced": {"POD_ATTN_POLICY": "balanced"},
+    "decode_first": {"POD_ATTN_POLICY": "decode_first"},
+    "proportional_global_ticket": {"POD_ATTN_POLICY": "proportional", "POD_ATTN_SMID_AWARE": "0"},
+}
+
+
+def run_sweep(args, rank, world, local):
+    """One JSON line per (workload, variant): FUSED, SERIAL and TWO_STREAM
+    mean us (L2 flushed before every call, CUDA events), the plan, and the
+    fused roofline fraction."""
+    from hybrid_prefill_decode_pod_b200 import pod_attn as pa
+    if rank != 0:
+        return 0
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks, _ = load_peaks()
+    stream = torch.cuda.current_stream(dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device=dev)
+    if args.sweep == "chunked16k":
+        points = [int(x) for x in args.sweep_points.split(",")] if args.sweep_points else \
+            [0, 4, 8, 12, 16, 20, 24, 28, 29, 30, 31]
+        workloads = ["chunked16k_%d" % i for i in points]
+        variants = SWEEP_VARIANTS
+    else:  # policies on the full-size configurations
+        workloads = args.sweep_points.split(",") if args.sweep_points else \
+            ["llama3_8b", "decode_heavy", "long_context", "paged"]
+        variants = SWEEP_POLICIES
+    for name in workloads:
+        batch = W.make_batch(W.get_config(name))
+        db = pa.DeviceBatch(batch, device=dev)
+        F, B, t_star, bound, _ = roofline_bound(batch, peaks)
+        for vname, env in variants.items():
+            old = {k: os.environ.get(k) for k in env}
+            os.environ.update(env)
+            try:
+                pod = pa.context_for(batch, device=local)
+            finally:
+                for k, v in old.items():
+                    if v is None:
+                        os.environ.pop(k, None)
+                    else:
+                        os.environ[k] = v
+            pre, dec = db.args(pod)
+            t = time_modes(pa, pod, pre, dec, stream, flush, args.steps, max(3, args.warmup))
+            pod.hybrid(pre, dec, pa.MODE_FUSED, stream)
+            plan = pod.last_plan()
+            st = pod.status(stream)
+            pod.close()
+            line = {"sweep": args.sweep, "workload": name, "variant": vname, "env": env,
+                    "fused_us": t["fused"], "serial_us": t["serial"],
+                    "two_stream_us": t["two_stream"],
+                    "speedup_vs_serial": t["serial"] / t["fused"],
+                    "speedup_vs_two_stream": t["two_stream"] / t["fused"],
+                    "t_star_us": t_star, "bound": bound,
+                    "fused_roofline_frac": t_star / t["fused"], "plan": plan, "status": st,
+                    "steps": args.steps}
+            print(json.dumps(line), flush=True)
+            if st != pa.POD_OK:
+                return 1
+        del db
+        torch.cuda.empty_cache()
+    return 0
+
+
 def run_e2e(pa, pod, batch, db, dev, stream, steps, flush):
     """Same metric through the C ABI with inputs in pinned host memory: every
     step copies Q and all K/V (or the pool and block tables) host -> device,
@@ -533,6 +614,11 @@ def main():
                     help="skip the other full-size configurations")
     ap.add_argument("--extra-steps", type=int, default=10)
     ap.add_argument("--stats", action="store_true")
+    ap.add_argument("--sweep", default=None, choices=["chunked16k", "policies"],
+                    help="ablation sweeps: the chunked 16K prompt (split limit, prefill tile) "
+                         "or the fused kernel's role policies; one JSON line per point")
+    ap.add_argument("--sweep-points", default=None,
+                    help="chunk indices (chunked16k) or workload names (policies), comma-separated")
     ap.add_argument("--only", default=None,
                     choices=["fused", "serial", "two_stream", "prefill_only", "decode_only"],
                     help="time one mode alone (profiler captures); prints a short JSON line")
@@ -543,6 +629,8 @@ def main():
     try:
         if args.impl == "reference":
             return run_reference(args, rank, world)
+        if args.sweep:
+            return run_sweep(args, rank, world, local)
         return run_gpu(args, rank, world, local)
     finally:
         if world > 1:

@@ -88,6 +88,7 @@ struct pod_attn_ctx {
   int dec_turn = 1;      // decode units each warp claims per decode turn of a fused CTA
   int dec_split = 0;     // 0: cost model; else keys per decode split (multiple of 16)
   int pre_split = 0;     // 0: makespan model; else KV splits per prefill tile
+  bool split_uncapped = false;  // forced splits ignore the two-wave cap (ablation)
   // prefill tile: a CTA pair on two SMs (M = 256, head_dim 128) or one SM
   bool use_pair = false;
   int pair_clusters = 0;  // clusters of two CTAs resident at once (pair kernel)
@@ -326,7 +327,7 @@ int build_plan(pod_attn_ctx* c, const pod_prefill_args* pa, const pod_decode_arg
   };
   if (n_draft > 0 && c->pre_split > 0) {
     int s_all = c->pre_split;
-    while (s_all > 1 && (long long)n_draft * s_all > 2LL * slots) --s_all;
+    while (!c->split_uncapped && s_all > 1 && (long long)n_draft * s_all > 2LL * slots) --s_all;
     for (int u = 0; u < n_draft; ++u) split[u] = std::min(s_all, max_split_of(u));
     if (!fits(split)) split.assign(n_draft, 1);
   } else if (n_draft > 0) {
@@ -693,6 +694,10 @@ void size_context(pod_attn_ctx* c) {
   c->cap_pgroups =
       (int)std::min<long long>(std::min<long long>(qtiles * c->H, 2LL * slots), 1 << 24);
   c->cap_pslots = 4 * slots;  // units x splits <= 2 slots, two query tiles per unit
+  if (c->split_uncapped) {     // forced splits past two waves (an ablation lever)
+    c->cap_pgroups = (int)std::min<long long>(qtiles * c->H, 1 << 20);
+    c->cap_pslots = (int)std::min<long long>(qtiles * c->H * kMaxPrefillSplit, 1 << 20);
+  }
   c->cap_pgroups = std::max(c->cap_pgroups, 1);
   c->cap_dreqs = std::max(cfg->max_decode_reqs, 1);
   c->cap_dunits =
@@ -772,7 +777,12 @@ int pod_attn_create(pod_attn_ctx** out, const pod_attn_config* cfg) {
   if (const char* e = std::getenv("POD_ATTN_SMID_AWARE")) c->smid_aware = std::atoi(e) != 0;
   if (const char* e = std::getenv("POD_ATTN_DEC_TURN")) c->dec_turn = std::max(1, std::atoi(e));
   if (const char* e = std::getenv("POD_ATTN_PREFILL_SPLIT"))
-    c->pre_split = std::max(0, std::min(kMaxPrefillSplit, std::atoi(e)));
+  {
+    // a negative count forces that many splits without the two-wave cap
+    const int v = std::atoi(e);
+    c->split_uncapped = v < 0;
+    c->pre_split = std::max(0, std::min(kMaxPrefillSplit, v < 0 ? -v : v));
+  }
   if (const char* e = std::getenv("POD_ATTN_DEC_SPLIT"))
     c->dec_split = std::max(0, std::atoi(e)) / kDecTile * kDecTile;
   // The CTA-pair prefill tile (head_dim 128) unless switched off; its
