@@ -85,6 +85,16 @@ struct PairLayout {
   static constexpr uint32_t T_O = 0, T_P = 128, T_S = 256;
 };
 
+// Pairs (of every 8) of the pair softmax's exponentials evaluated by
+// exp2_poly2 on the FMA pipe instead of ex2 on MUFU, on tiles without masked
+// keys. Per SM and KV tile the MMAs take 1024 tensor-core cycles and the
+// 16384 exponentials 1024 MUFU cycles (16 per clock per SM), so moving a
+// share off MUFU keeps it from setting the pace.
+#ifndef POD_PAIR_POLY_PAIRS
+#define POD_PAIR_POLY_PAIRS 0
+#endif
+constexpr int kPairPolyPairs = POD_PAIR_POLY_PAIRS;
+
 // misc[] words of the pair kernel
 constexpr int kMiscTmem = 0, kMiscRole = 1, kMiscUnit = 2, kMiscAbort = 3, kMiscPEmpty = 5,
               kMiscDEmpty = 6, kMiscPending = 7, kMiscMerge = 8, kMiscMbRole = 10,
@@ -399,8 +409,16 @@ POD_DEV bool pair_softmax(const Plan& P, const PrefillRange& pr, int rank, uint8
     for (int c = 0; c < 32; ++c) {
       float x0, x1;
       f2_unpack(ffma2(f2_pack(s[2 * c], s[2 * c + 1]), sc2, nm2), x0, x1);
-      const float p0 = ex2(x0), p1 = ex2(x1);
-      const uint64_t p2 = f2_pack(p0, p1);
+      float p0, p1;
+      uint64_t p2;
+      if (!masked_tile && (c & 7) >= 8 - kPairPolyPairs) {
+        p2 = exp2_poly2(x0, x1);
+        f2_unpack(p2, p0, p1);
+      } else {
+        p0 = ex2(x0);
+        p1 = ex2(x1);
+        p2 = f2_pack(p0, p1);
+      }
       pk[c] = pack_bf16(p0, p1);
       acc[c & 3] = (c < 4) ? p2 : fadd2(acc[c & 3], p2);
     }

@@ -84,6 +84,26 @@ PROBE_CONFIGS = {
     "long_context_probe": HybridConfig(
         "long_context_probe", 64, 8, 128, prefill=((4096, 1024),), decode_ctx=(4096,) * 16),
 }
+# Variants of the pages' model shapes (the summary's §A.2 / §A.3.5 list
+# Llama-2-7B, Llama-3-8B and Yi-6B; their attention shapes are those of the
+# public model architectures: Llama-2-7B is multi-head, 32 heads of 128;
+# Yi-6B groups 32 query heads over 4 KV heads of 128), a head_dim-64 mix, and
+# a batch of many small chunks, each beside 64 decodes at context 4096.
+VARIANT_CONFIGS = {
+    "llama2_7b_mha": HybridConfig(
+        "llama2_7b_mha", 32, 32, 128, prefill=((4096, 512),), decode_ctx=(4096,) * 64),
+    "yi6b_g8": HybridConfig(
+        "yi6b_g8", 32, 4, 128, prefill=((4096, 512),), decode_ctx=(4096,) * 64),
+    "d64_mix": HybridConfig(
+        "d64_mix", 16, 4, 64, prefill=((4096, 512),), decode_ctx=(4096,) * 64),
+    # 16 chunks (the per-call maximum) of 1..40 tokens after 0..8192 cached tokens
+    "many_chunks": HybridConfig(
+        "many_chunks", 32, 8, 128,
+        prefill=tuple(((2749 * i) % 8193, 1 + (37 * i) % 40) for i in range(16)),
+        decode_ctx=(4096,) * 64),
+}
+PROBE_CONFIGS.update(VARIANT_CONFIGS)
+
 # Chunked prefill of a 16K-token prompt in chunks of 512 beside 64 decodes at the
 # same context (the paper's per-chunk study of a long prompt, restated on
 # synthetic Llama-3-8B-shaped inputs): point i has prior 512 i and decodes at
@@ -101,6 +121,10 @@ CONFIG_DESCRIPTIONS = {
     "long_context": "long-context 70B-like: 64 q / 8 kv heads, d 128; 1 prefill chunk 1024 after prior 16384 + 16 decodes U[16384, 32768]",
     "paged": "paged-KV: 32 q / 8 kv heads, d 128; 2 prefill chunks of 512 (priors 2048, 8192) + 128 decodes U[1024, 16384], 16-token blocks, permuted",
     "long_context_probe": "profiling probe: 64 q / 8 kv heads, d 128; 1 prefill chunk 1024 after prior 4096 + 16 decodes at 4096",
+    "llama2_7b_mha": "Llama-2-7B-shaped (multi-head): 32 q / 32 kv heads, d 128; 1 prefill chunk 512 after prior 4096 + 64 decodes at 4096",
+    "yi6b_g8": "Yi-6B-shaped: 32 q / 4 kv heads, d 128; 1 prefill chunk 512 after prior 4096 + 64 decodes at 4096",
+    "d64_mix": "head_dim 64: 16 q / 4 kv heads, d 64; 1 prefill chunk 512 after prior 4096 + 64 decodes at 4096",
+    "many_chunks": "16 prefill chunks of 1-40 tokens after 0-8192 cached tokens + 64 decodes at 4096; 32 q / 8 kv heads, d 128",
     **{"chunked16k_%d" % i: "chunk %d of a 16K prompt: 32 q / 8 kv heads, d 128; prefill chunk 512 after prior %d + 64 decodes at %d" % (i, 512 * i, 512 * (i + 1)) for i in range(32)},
 }
 

@@ -181,33 +181,55 @@ typedef struct {
 
 /* Validates cfg, allocates the workspace on cfg->device. *out is set on
  * success only. Returns POD_OK, POD_EINVAL, POD_EUNSUPPORTED, POD_ENOMEM or
- * POD_ECUDA. */
+ * POD_ECUDA.
+ * Follows: the fused kernel is sized for whichever phase needs more shared
+ * memory (POD-Attention summary §4.3 "Implementing CTA-parallel Fusion"), and
+ * its split prefill and virtual decode units write partial results that a
+ * merge combines (§4.2.3 "Virtual Decode CTAs"): every buffer for those is
+ * allocated here, once. The create-time caps bound what one call admits
+ * (Silicon & Systems digest, "Isolation and predictability"). */
 POD_API int pod_attn_create(pod_attn_ctx** out, const pod_attn_config* cfg);
 
 /* One hybrid batch. Either argument may be NULL or have num_reqs == 0.
- * mode is a pod_mode. stream is a cudaStream_t. */
+ * mode is a pod_mode. stream is a cudaStream_t.
+ * Follows: a hybrid batch of prefill chunks and decodes (POD-Attention summary
+ * §2.1 "Large Language Model (LLM) Inference") computed by one fused kernel
+ * (§4 "POD-Attention", §4.4 persistent form), or by the separate-kernel
+ * baselines FA_Serial and FA_Streams (§3.2 "Analysis of Readily Available
+ * Methods"). Returns POD_OK, POD_EINVAL, POD_ECAPACITY or POD_ECUDA before
+ * or at enqueue time; device problems go to the status word. */
 POD_API int pod_attn_hybrid(pod_attn_ctx* ctx, const pod_prefill_args* prefill,
                     const pod_decode_args* decode, int mode, void* stream);
 
-/* Prefill requests alone (the persistent launch with no decode work). */
+/* Prefill requests alone (the persistent launch with no decode work): the
+ * compute-bound phase of the summary's §2.1, as the serial baseline runs it
+ * (§3.2). Errors as for pod_attn_hybrid. */
 POD_API int pod_attn_prefill_only(pod_attn_ctx* ctx, const pod_prefill_args* prefill, void* stream);
 
-/* Decode requests alone (split-KV decode launch + LSE merge launch). */
+/* Decode requests alone (split-KV decode launch + LSE merge launch): the
+ * memory-bound phase of the summary's §2.1, in one-warp units with a
+ * 16-key tile (§4.2.1 "Tile Sizes", §4.2.3 "Virtual Decode CTAs"). Errors as
+ * for pod_attn_hybrid. */
 POD_API int pod_attn_decode_only(pod_attn_ctx* ctx, const pod_decode_args* decode, void* stream);
 
 /* Synchronises `stream`, then returns and clears the sticky device status
- * (POD_OK or POD_ETIMEOUT), or POD_ECUDA if the synchronisation failed. */
+ * (POD_OK or POD_ETIMEOUT), or POD_ECUDA if the synchronisation failed.
+ * (No counterpart in the pages: the failure signal of the digest's
+ * "Isolation and predictability".) */
 POD_API int pod_attn_status(pod_attn_ctx* ctx, void* stream);
 
-/* Planner decisions of the last call. */
+/* Planner decisions of the last call: split counts, the prefill tile, the
+ * role ratio (the summary's §4.2.2, §4.2.3 and §5.4). POD_EINVAL on NULL. */
 POD_API int pod_attn_last_plan(const pod_attn_ctx* ctx, pod_plan_info* out);
 
 /* Synchronises `stream` and reads the per-SM role counters of the last call
- * (requires POD_FLAG_STATS at create, else POD_EINVAL). */
+ * (requires POD_FLAG_STATS at create, else POD_EINVAL): which SMs ran both
+ * prefill and decode work (the co-location of the summary's §4.1). */
 POD_API int pod_attn_get_stats(pod_attn_ctx* ctx, void* stream, pod_stats* out);
 
 /* Synchronises the device, reads the sticky status, frees everything.
- * Returns that status (POD_OK or POD_ETIMEOUT) or POD_ECUDA. NULL is a no-op. */
+ * Returns that status (POD_OK or POD_ETIMEOUT) or POD_ECUDA. NULL is a no-op.
+ * (Resource release; no counterpart in the pages.) */
 POD_API int pod_attn_destroy(pod_attn_ctx* ctx);
 
 /* ---------------------------------------------------------------------------

@@ -247,14 +247,19 @@ def _full_ref(name):
     per test session: the oracle is the expensive side)."""
     if name not in _FULL_REF:
         _FULL_REF.clear()  # keep one configuration's tensors alive at a time
-        b = W.make_batch(W.CONFIGS[name])
+        b = W.make_batch(W.get_config(name))
         _FULL_REF[name] = (b, oracle.hybrid(b))
     return _FULL_REF[name]
 
 
 FULL_SIZE = [("llama3_8b", "fused"), ("decode_heavy", "fused"),
              ("long_context", "fused"), ("long_context", "serial"), ("long_context", "two_stream"),
-             ("paged", "fused"), ("paged", "serial"), ("paged", "two_stream")]
+             ("paged", "fused"), ("paged", "serial"), ("paged", "two_stream"),
+             # shape variants: multi-head, group of 8, head_dim 64, 16 small chunks
+             ("llama2_7b_mha", "fused"), ("yi6b_g8", "fused"), ("d64_mix", "fused"),
+             ("many_chunks", "fused"), ("many_chunks", "serial"),
+             # a late chunk of the chunked 16K prompt (prior 15872 + 512, 64 decodes)
+             ("chunked16k_31", "fused")]
 
 
 @pytest.mark.slow
