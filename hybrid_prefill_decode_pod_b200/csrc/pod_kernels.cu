@@ -792,8 +792,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
           if (lane == 0) pair_producer<D>(P, T, pr, rank, sm, ps, pa);
           __syncwarp();
         }
-      } else {
-        // decode turn: each role warp claims up to dec_turn units; once every
+      } else if (warp < L::TURN_WARPS) {
+        // decode turn: each turn warp claims up to dec_turn units; once every
         // prefill unit has been claimed it keeps claiming until the decode
         // queue is empty. The peer also ends its turn when the leader has
         // posted a new decision (the pair is wanted for a prefill unit).
@@ -833,7 +833,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       }
       if (!decode_unit_warp<D, L::SIDE_DEC_ST>(
               P, u, sm + L::SIDE_OFF + sw * L::SIDE_DEC_WARP,
-              bars + (L::B_DEC + kRoleWarps * L::ROLE_DEC_ST + sw * L::SIDE_DEC_ST) * 8, side_ring,
+              bars + (L::B_DEC + L::TURN_WARPS * L::ROLE_DEC_ST + sw * L::SIDE_DEC_ST) * 8, side_ring,
               lane, true, abort_flag))
         break;
     }

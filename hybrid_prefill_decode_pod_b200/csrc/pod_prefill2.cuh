@@ -49,11 +49,16 @@ struct PairLayout {
   static constexpr int PREFILL_END = V_OFF + VS * VH;
   static constexpr int DEC_ROW = D * 2 + 16;             // padded row: conflict-free ldmatrix
   static constexpr int DEC_STAGE = 2 * kDecTile * DEC_ROW;
-  static constexpr int ROLE_DEC_ST = 2;                  // ring depth of a role warp's decode turn
-  static constexpr int SIDE_DEC_ST = 3;                  // ring depth of a side decode warp
+  // Decode turns run on the 8 softmax warps (the MMA and producer warps sit
+  // them out); their 2-stage rings overlay the prefill rings. The side
+  // warps' deeper rings lie beyond both, so every SM keeps 80 KB of decode
+  // K/V loads in flight beside a prefill unit.
+  static constexpr int TURN_WARPS = kSoftmaxWarps;
+  static constexpr int ROLE_DEC_ST = 2;                  // ring depth of a decode-turn warp
+  static constexpr int SIDE_DEC_ST = 5;                  // ring depth of a side decode warp
   static constexpr int ROLE_DEC_WARP = ROLE_DEC_ST * DEC_STAGE;
   static constexpr int SIDE_DEC_WARP = SIDE_DEC_ST * DEC_STAGE;
-  static constexpr int DEC_END = kRoleWarps * ROLE_DEC_WARP;  // decode turns overlay prefill
+  static constexpr int DEC_END = TURN_WARPS * ROLE_DEC_WARP;  // decode turns overlay prefill
   static constexpr int SIDE_OFF = PREFILL_END > DEC_END ? PREFILL_END : DEC_END;
   static constexpr int XCH_OFF = SIDE_OFF + kSideDecWarps * SIDE_DEC_WARP;
   // row max of the two column halves, double-buffered by KV tile parity, then
@@ -75,7 +80,7 @@ struct PairLayout {
   static constexpr int B_MB = B_OR + 1;           // peer: the leader posted a claim
   static constexpr int B_ACK = B_MB + 1;          // leader: the peer read the claim
   static constexpr int B_DEC = B_ACK + 1;         // decode rings: role warps, then side warps
-  static constexpr int N_BARS = B_DEC + kRoleWarps * ROLE_DEC_ST + kSideDecWarps * SIDE_DEC_ST;
+  static constexpr int N_BARS = B_DEC + TURN_WARPS * ROLE_DEC_ST + kSideDecWarps * SIDE_DEC_ST;
   static constexpr int MISC_OFF = BAR_OFF + N_BARS * 8;
   static constexpr int TOTAL = MISC_OFF + 64;
   static_assert(TOTAL <= 227 * 1024, "pair CTA exceeds the shared memory of an SM");
@@ -94,6 +99,15 @@ struct PairLayout {
 #define POD_PAIR_POLY_PAIRS 0
 #endif
 constexpr int kPairPolyPairs = POD_PAIR_POLY_PAIRS;
+
+// The softmax warps' hand-offs to the leader's MMA thread (S read, P
+// written) are tensor-memory hand-offs ordered by tcgen05 fences around the
+// barrier: by default a plain remote arrival and wait, as for shared-memory
+// stages; POD_PAIR_ACQREL_CLUSTER=1 makes them cluster-scope release /
+// acquire (measured slower, kept for comparison).
+#ifndef POD_PAIR_ACQREL_CLUSTER
+#define POD_PAIR_ACQREL_CLUSTER 0
+#endif
 
 // misc[] words of the pair kernel
 constexpr int kMiscTmem = 0, kMiscRole = 1, kMiscUnit = 2, kMiscAbort = 3, kMiscPEmpty = 5,
@@ -139,6 +153,21 @@ POD_DEV bool pwait_c(uint32_t bar, uint32_t parity, const Plan& P, const PairAbo
       return false;
     }
   }
+}
+// The MMA thread's wait for the softmax warps' hand-offs.
+POD_DEV bool pwait_handoff(uint32_t bar, uint32_t parity, const Plan& P, const PairAbort& pa) {
+#if POD_PAIR_ACQREL_CLUSTER
+  return pwait_c(bar, parity, P, pa);
+#else
+  return pwait(bar, parity, P, pa);
+#endif
+}
+POD_DEV void handoff_arrive(uint32_t cluster_addr) {
+#if POD_PAIR_ACQREL_CLUSTER
+  mbar_arrive_cluster(cluster_addr);
+#else
+  mbar_arrive_remote(cluster_addr);
+#endif
 }
 POD_DEV bool pwait_warp(uint32_t bar, uint32_t parity, const Plan& P, const PairAbort& pa) {
   const bool ok = pwait(bar, parity, P, pa);
@@ -252,7 +281,8 @@ POD_DEV bool pair_mma(const Plan& P, const PrefillRange& pr, uint8_t* sm, uint32
     const uint32_t st = it % L::KS, ph = (it / L::KS) & 1;
     if (!pwait(bars + (L::B_KF + st) * 8, ph, P, pa)) return false;
     // S_b last held S_{it-2}: every softmax warp of both CTAs has read it
-    if (it >= 2 && !pwait_c(bars + (L::B_SE + b) * 8, ((it - 2) >> 1) & 1, P, pa)) return false;
+    if (it >= 2 && !pwait_handoff(bars + (L::B_SE + b) * 8, ((it - 2) >> 1) & 1, P, pa))
+      return false;
     tc_fence_after();
     const uint64_t kd = dk0 + (uint64_t)(st * (L::KH >> 4));
 #pragma unroll
@@ -274,7 +304,7 @@ POD_DEV bool pair_mma(const Plan& P, const PrefillRange& pr, uint8_t* sm, uint32
     const uint32_t it = ps.kv + j, b = it & 1;
     const uint32_t st = it % L::VS, ph = (it / L::VS) & 1;
     if (!pwait(bars + (L::B_VF + st) * 8, ph, P, pa)) return false;
-    if (!pwait_c(bars + (L::B_PF + b) * 8, (it >> 1) & 1, P, pa)) return false;
+    if (!pwait_handoff(bars + (L::B_PF + b) * 8, (it >> 1) & 1, P, pa)) return false;
     tc_fence_after();
     const uint64_t vd = dv0 + (uint64_t)(st * (L::VH >> 4));
     const uint32_t pcol = tmem + L::T_P + 64 * b;
@@ -348,7 +378,7 @@ POD_DEV bool pair_softmax(const Plan& P, const PrefillRange& pr, int rank, uint8
       // S_b may be overwritten once every softmax warp of both CTAs has it
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(lbars + (L::B_SE + b) * 8);
+      if (lane == 0) handoff_arrive(lbars + (L::B_SE + b) * 8);
       if (masked_tile) {
         const int k0 = tile0 + 64 * hf;
 #pragma unroll
@@ -438,7 +468,7 @@ POD_DEV bool pair_softmax(const Plan& P, const PrefillRange& pr, int rank, uint8
     tmem_st32(tmem + lane_base + L::T_P + 64 * b + 32 * hf, pk);  // waits for the store
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive_cluster(lbars + (L::B_PF + b) * 8);
+    if (lane == 0) handoff_arrive(lbars + (L::B_PF + b) * 8);
   }
   // O complete
   if (!failed) {

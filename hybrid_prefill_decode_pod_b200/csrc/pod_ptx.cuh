@@ -251,6 +251,13 @@ POD_DEV void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                : "memory");
 }
+// Arrive on a barrier given by its cluster address, default (CTA-scope
+// release) semantics: the hand-off a producer in one CTA gives a consumer in
+// the other when the data itself moves in another proxy (TMEM written by
+// tcgen05.st and ordered by tcgen05.fence, or shared memory refilled by TMA).
+POD_DEV void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
 // try_wait with cluster-scope acquire: for barriers the peer CTA's threads
 // arrive on, so their earlier writes are visible after the wait.
 POD_DEV uint32_t mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
