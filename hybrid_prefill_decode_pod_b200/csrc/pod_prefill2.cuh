@@ -109,6 +109,30 @@ constexpr int kPairPolyPairs = POD_PAIR_POLY_PAIRS;
 #define POD_PAIR_ACQREL_CLUSTER 0
 #endif
 
+// How the pair softmax rounds P to bf16 pairs: 0 cvt.rn.bf16x2 (the XU pipe,
+// which the exponentials also use), 1 round half away from zero with integer
+// adds (P >= 0; differs from nearest-even only on exact ties), 2 nearest even
+// with integer ops.
+#ifndef POD_PAIR_PACK
+#define POD_PAIR_PACK 1
+#endif
+POD_DEV uint32_t pair_pack(float lo, float hi) {
+#if POD_PAIR_PACK == 0
+  return pack_bf16(lo, hi);
+#elif POD_PAIR_PACK == 1
+  return pack_bf16_rha(lo, hi);
+#else
+  return pack_bf16_int(lo, hi);
+#endif
+}
+
+// K tiles the pair producer issues ahead of V tiles (0: K_j, V_j, K_j+1, ...).
+#ifndef POD_PAIR_K_LEAD
+#define POD_PAIR_K_LEAD 2
+#endif
+constexpr int kKLead = POD_PAIR_K_LEAD;
+static_assert(kKLead >= 0 && kKLead < 3, "the lead must leave a K stage for the next tile");
+
 // misc[] words of the pair kernel
 constexpr int kMiscTmem = 0, kMiscRole = 1, kMiscUnit = 2, kMiscAbort = 3, kMiscPEmpty = 5,
               kMiscDEmpty = 6, kMiscPending = 7, kMiscMerge = 8, kMiscMbRole = 10,
@@ -208,10 +232,14 @@ POD_DEV bool pair_producer(const Plan& P, const TmaDescs& T, const PrefillRange&
   const CUtensorMap* km = P.paged ? &T.k[0] : &T.k[pr.req];
   const CUtensorMap* vm = P.paged ? &T.v[0] : &T.v[pr.req];
   const int last_page = (R.kv_len - 1) >> 4;
-  for (int j = 0; j < pr.n; ++j) {
-    const uint32_t it = ps.kv + j;
-    const int key0 = (pr.t0 + j) * kKVTile;
-    {  // K half: keys key0 + 64 rank .. +63, every column (two 64-column blocks)
+  // K tiles are issued kKLead tiles ahead of V tiles: the MMA order needs
+  // K_{j+2} (for S_{j+2}) before V_j (for P_j V_j), and a V stage is freed
+  // only by a P V, which waits for the softmax.
+  for (int t = 0; t < pr.n + kKLead; ++t) {
+    const int j = t;  // K tile of this step
+    if (j < pr.n) {  // K half: keys key0 + 64 rank .. +63, every column (two 64-column blocks)
+      const uint32_t it = ps.kv + j;
+      const int key0 = (pr.t0 + j) * kKVTile;
       const uint32_t st = it % L::KS, ph = (it / L::KS) & 1;
       if (it >= (uint32_t)L::KS && !pwait(bars + (L::B_KE + st) * 8, ph ^ 1, P, pa)) return false;
       const uint32_t full = lbars + (L::B_KF + st) * 8;
@@ -230,7 +258,10 @@ POD_DEV bool pair_producer(const Plan& P, const TmaDescs& T, const PrefillRange&
       }
       ps.kissued = it + 1;
     }
-    {  // V half: keys key0 .. +127, columns 64 rank .. +63 (one 64-column block)
+    if (t - kKLead >= 0) {  // V half: keys key0 .. +127, columns 64 rank .. +63 (one block)
+      const int jv = t - kKLead;
+      const uint32_t it = ps.kv + jv;
+      const int key0 = (pr.t0 + jv) * kKVTile;
       const uint32_t st = it % L::VS, ph = (it / L::VS) & 1;
       if (it >= (uint32_t)L::VS && !pwait(bars + (L::B_VE + st) * 8, ph ^ 1, P, pa)) return false;
       const uint32_t full = lbars + (L::B_VF + st) * 8;
@@ -449,7 +480,7 @@ POD_DEV bool pair_softmax(const Plan& P, const PrefillRange& pr, int rank, uint8
         p1 = ex2(x1);
         p2 = f2_pack(p0, p1);
       }
-      pk[c] = pack_bf16(p0, p1);
+      pk[c] = pair_pack(p0, p1);
       acc[c & 3] = (c < 4) ? p2 : fadd2(acc[c & 3], p2);
     }
     float lt;
