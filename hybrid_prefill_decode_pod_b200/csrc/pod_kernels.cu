@@ -51,6 +51,13 @@ constexpr int kSoftPairs = POD_SOFT_EXP2_PAIRS;
 #define POD_PACK(a, b) pack_bf16(a, b)
 #endif
 
+// L2 cache-policy hints on the bulk loads: prefill K/V evict-last (several
+// query tiles re-read each tile), decode K/V evict-first (read once), so the
+// decode stream of a fused launch does not push the prefill's tiles out of L2.
+#ifndef POD_L2_HINTS
+#define POD_L2_HINTS 1
+#endif
+
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kStatusTimeout = -5;
@@ -299,6 +306,9 @@ POD_DEV bool decode_unit_warp(const Plan& P, int u, uint8_t* wsm, uint32_t bar0,
   const uint16_t* kbase = P.paged ? P.k_pool : R.k;
   const uint16_t* vbase = P.paged ? P.v_pool : R.v;
   const uint32_t wsm_a = smem_u32(wsm);
+#if POD_L2_HINTS
+  const uint64_t once = l2_evict_first();  // decode K/V is read once
+#endif
 
   auto issue = [&](int t) {
     const uint32_t it = ring + t;
@@ -311,7 +321,11 @@ POD_DEV bool decode_unit_warp(const Plan& P, int u, uint8_t* wsm, uint32_t bar0,
     const size_t off = row_off(key);
     const uint16_t* src = (lane < 16) ? (kbase + off) : (vbase + off);
     const uint32_t dst = wsm_a + st * STAGE + (lane < 16 ? 0 : kDecTile * ROW) + (lane & 15) * ROW;
+#if POD_L2_HINTS
+    bulk_load_hint(dst, src, D * 2, bar, once);
+#else
     bulk_load(dst, src, D * 2, bar);
+#endif
   };
 
   fence_proxy_async_smem();

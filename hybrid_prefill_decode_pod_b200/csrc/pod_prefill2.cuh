@@ -232,6 +232,12 @@ POD_DEV bool pair_producer(const Plan& P, const TmaDescs& T, const PrefillRange&
   const CUtensorMap* km = P.paged ? &T.k[0] : &T.k[pr.req];
   const CUtensorMap* vm = P.paged ? &T.v[0] : &T.v[pr.req];
   const int last_page = (R.kv_len - 1) >> 4;
+#if POD_L2_HINTS
+  const uint64_t keep = l2_evict_last();  // K/V tiles are re-read by other query tiles
+#define POD_PAIR_LOAD(d, m, f, x, y, z) tma_load_3d_pair_hint(d, m, f, x, y, z, keep)
+#else
+#define POD_PAIR_LOAD(d, m, f, x, y, z) tma_load_3d_pair(d, m, f, x, y, z)
+#endif
   // K tiles are issued kKLead tiles ahead of V tiles: the MMA order needs
   // K_{j+2} (for S_{j+2}) before V_j (for P_j V_j), and a V stage is freed
   // only by a P V, which waits for the softmax.
@@ -247,13 +253,13 @@ POD_DEV bool pair_producer(const Plan& P, const TmaDescs& T, const PrefillRange&
       const uint32_t dst = base + L::K_OFF + st * L::KH;
       const int k0 = key0 + 64 * rank;
       if (!P.paged) {
-        for (int b = 0; b < NB; ++b) tma_load_3d_pair(dst + b * (64 * 128), km, full, 64 * b, g, k0);
+        for (int b = 0; b < NB; ++b) POD_PAIR_LOAD(dst + b * (64 * 128), km, full, 64 * b, g, k0);
       } else {
         for (int pg = 0; pg < 4; ++pg) {
           const int lp = min((k0 >> 4) + pg, last_page);
           const int phys = __ldg(P.bt_p + (size_t)R.bt_row * P.bt_stride_p + lp);
           for (int b = 0; b < NB; ++b)
-            tma_load_3d_pair(dst + b * (64 * 128) + pg * 16 * 128, km, full, 64 * b, g, phys * 16);
+            POD_PAIR_LOAD(dst + b * (64 * 128) + pg * 16 * 128, km, full, 64 * b, g, phys * 16);
         }
       }
       ps.kissued = it + 1;
@@ -268,12 +274,12 @@ POD_DEV bool pair_producer(const Plan& P, const TmaDescs& T, const PrefillRange&
       if (rank == 0) mbar_expect_tx(bars + (L::B_VF + st) * 8, 2 * L::VH);
       const uint32_t dst = base + L::V_OFF + st * L::VH;
       if (!P.paged) {
-        tma_load_3d_pair(dst, vm, full, 64 * rank, g, key0);
+        POD_PAIR_LOAD(dst, vm, full, 64 * rank, g, key0);
       } else {
         for (int pg = 0; pg < kKVTile / 16; ++pg) {
           const int lp = min((key0 >> 4) + pg, last_page);
           const int phys = __ldg(P.bt_p + (size_t)R.bt_row * P.bt_stride_p + lp);
-          tma_load_3d_pair(dst + pg * 16 * 128, vm, full, 64 * rank, g, phys * 16);
+          POD_PAIR_LOAD(dst + pg * 16 * 128, vm, full, 64 * rank, g, phys * 16);
         }
       }
       ps.vissued = it + 1;
@@ -281,6 +287,7 @@ POD_DEV bool pair_producer(const Plan& P, const TmaDescs& T, const PrefillRange&
   }
   ps.kv += pr.n;
   return true;
+#undef POD_PAIR_LOAD
 }
 
 // ---- MMA issuer (one thread of the leader CTA). Order per unit:
