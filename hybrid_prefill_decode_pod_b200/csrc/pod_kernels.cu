@@ -702,7 +702,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     for (int i = 0; i < L::N_BARS; ++i) {
       uint32_t cnt = 1;
       if (i == L::B_SE || i == L::B_SE + 1 || i == L::B_PF || i == L::B_PF + 1)
-        cnt = 2 * kSoftmaxWarps;  // every softmax warp of both CTAs
+        cnt = 2 * kTileOwners;  // the tile's owner warps in both CTAs
       mbar_init(bars + i * 8, cnt);
     }
     fence_mbar_init();

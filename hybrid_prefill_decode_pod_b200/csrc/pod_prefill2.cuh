@@ -61,8 +61,8 @@ struct PairLayout {
   static constexpr int DEC_END = TURN_WARPS * ROLE_DEC_WARP;  // decode turns overlay prefill
   static constexpr int SIDE_OFF = PREFILL_END > DEC_END ? PREFILL_END : DEC_END;
   static constexpr int XCH_OFF = SIDE_OFF + kSideDecWarps * SIDE_DEC_WARP;
-  // row max of the two column halves, double-buffered by KV tile parity, then
-  // the two halves' row sums: float [2][2][128] + [2][128]
+  // the handed-on reference max [2][128], then the final references and
+  // row-sum shares [2][128] + [2][128]
   static constexpr int XCH_BYTES = 6 * kQTile * 4;
   static constexpr int BAR_OFF = (XCH_OFF + XCH_BYTES + 127) & ~127;
   // barrier indices
@@ -73,8 +73,8 @@ struct PairLayout {
   static constexpr int B_VF = B_KE + KS;          // V tile landed (leader) [VS]
   static constexpr int B_VE = B_VF + VS;          // V stage read by its P V MMA [VS]
   static constexpr int B_SF = B_VE + VS;          // S_b in TMEM [2]
-  static constexpr int B_SE = B_SF + 2;           // S_b read by all 16 softmax warps (leader) [2]
-  static constexpr int B_PF = B_SE + 2;           // P_b written by all 16 softmax warps (leader) [2]
+  static constexpr int B_SE = B_SF + 2;           // S_b read by its 8 owner warps (leader) [2]
+  static constexpr int B_PF = B_SE + 2;           // P_b written by its 8 owner warps (leader) [2]
   static constexpr int B_PE = B_PF + 2;           // P_b V done: P_b free, O current [2]
   static constexpr int B_OR = B_PE + 2;           // O final for the unit
   static constexpr int B_MB = B_OR + 1;           // peer: the leader posted a claim
@@ -133,6 +133,16 @@ POD_DEV uint32_t pair_pack(float lo, float hi) {
 constexpr int kKLead = POD_PAIR_K_LEAD;
 static_assert(kKLead >= 0 && kKLead < 3, "the lead must leave a K stage for the next tile");
 
+// Named barriers of the pair kernel: 1 the role warps; per lane quarter q,
+// kBarHandoff0 + 2 q + h carries the reference max from the owner of tiles of
+// parity h to the other warp (one-way: arrive, then sync), kBarFinal0 + q the
+// two warps' final exchange; kBarSoftmaxAll all eight softmax warps.
+constexpr int kBarHandoff0 = 2;    // 2 .. 9
+constexpr int kBarFinal0 = 10;     // 10 .. 13
+constexpr int kBarSoftmaxAll = 14;
+// softmax warps that read each S tile and write each P tile (per CTA)
+constexpr int kTileOwners = kSoftmaxWarps / 2;
+
 // misc[] words of the pair kernel
 constexpr int kMiscTmem = 0, kMiscRole = 1, kMiscUnit = 2, kMiscAbort = 3, kMiscPEmpty = 5,
               kMiscDEmpty = 6, kMiscPending = 7, kMiscMerge = 8, kMiscMbRole = 10,
@@ -151,18 +161,23 @@ POD_DEV void pair_raise_abort(const Plan& P, const PairAbort& pa) {
   st_cluster_u32(pa.peer_flag, 1u);
 }
 
-// Bounded wait for a TMA / MMA-commit barrier of this CTA.
-POD_DEV bool pwait(uint32_t bar, uint32_t parity, const Plan& P, const PairAbort& pa) {
-  if (mbar_try_wait(bar, parity)) return true;
+// Bounded wait for a TMA / MMA-commit barrier of this CTA: one try inline,
+// the spinning slow path out of line (it keeps the hot loops' registers free).
+__device__ __noinline__ bool pwait_slow(uint32_t bar, uint32_t parity, const Plan& P,
+                                        volatile int* flag, uint32_t peer_flag) {
   const long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (*pa.flag) return false;
+    if (*flag) return false;
     if (clock64() - t0 > P.wait_budget) {
-      pair_raise_abort(P, pa);
+      pair_raise_abort(P, PairAbort{flag, peer_flag});
       return false;
     }
   }
+}
+POD_DEV bool pwait(uint32_t bar, uint32_t parity, const Plan& P, const PairAbort& pa) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return pwait_slow(bar, parity, P, pa.flag, pa.peer_flag);
 }
 // Bounded wait for a barrier that threads of the other CTA arrive on
 // (cluster-scope acquire).
@@ -369,10 +384,16 @@ POD_DEV bool pair_mma(const Plan& P, const PrefillRange& pr, uint8_t* sm, uint32
   return true;
 }
 
-// ---- softmax + epilogue (warps 0-7 of each CTA). Every warp passes the same
-// named barriers the same number of times whatever happens (a failed wait
-// only skips tensor-memory work), so a timeout can never leave a barrier
-// short of arrivals.
+// ---- softmax + epilogue (warps 0-7 of each CTA). Warp w serves the rows of
+// its TMEM lane quarter, 32 (w % 4) .. +31, and the unit's KV tiles t with
+// t % 2 == w / 4, all 128 keys of each: the two warps of a lane quarter share
+// a sub-partition and work on consecutive tiles at the same time, so their
+// exponentials interleave on its MUFU unit. The lazily raised reference max
+// of the rows passes from the owner of tile t to the owner of tile t + 1
+// through shared memory under a one-way named barrier (arrive, then sync),
+// handed on before the exponentials. Every warp passes its named barriers the
+// same number of times whatever happens (a failed wait only skips
+// tensor-memory work), so a timeout can never leave a barrier short.
 template <int D>
 POD_DEV bool pair_softmax(const Plan& P, const PrefillRange& pr, int rank, uint8_t* sm,
                           uint32_t tmem, PairPipe& ps, int tid, const PairAbort& pa,
@@ -382,7 +403,7 @@ POD_DEV bool pair_softmax(const Plan& P, const PrefillRange& pr, int rank, uint8
   const uint32_t lbars = mapa_shared(bars, 0);
   const PrefillReq R = P.preq[pr.req];
   const int warp = tid >> 5, lane = tid & 31;
-  const int q4 = warp & 3, hf = warp >> 2;  // lane quarter, column half
+  const int q4 = warp & 3, hf = warp >> 2;  // lane quarter, tile parity
   const int row = q4 * 32 + lane;
   const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
   const int head = pr.head[rank], qtile = pr.qtile[rank];
@@ -391,119 +412,123 @@ POD_DEV bool pair_softmax(const Plan& P, const PrefillRange& pr, int rank, uint8
   const int lim = R.prior + q_local;               // last visible key (inclusive)
   const int mask_from = R.prior + qtile * kQTile;  // KV tiles ending above this need masking
   const float sc = P.scale_log2;
-  float* xmax = reinterpret_cast<float*>(sm + L::XCH_OFF);  // [2 parity][2 half][128]
-  float* xsum = xmax + 4 * kQTile;                          // [2 half][128]
-  const int pair_bar = 2 + q4;                              // warps q4 and q4 + 4
-  float m_run = -INFINITY, l_run = 0.f;
-  bool failed = false;  // warp-uniform
+  float* xref = reinterpret_cast<float*>(sm + L::XCH_OFF);  // [2 from][128] handed-on reference
+  float* xfin = xref + 2 * kQTile;                          // [2][128] m, then [2][128] l
+  const int hand_to = kBarHandoff0 + 2 * q4 + hf;           // this warp -> the other
+  const int hand_from = kBarHandoff0 + 2 * q4 + (hf ^ 1);   // the other -> this warp
+  const int n = pr.n;
+  float m_ref = -INFINITY;  // reference max (log2 units) O and l_h are scaled to
+  float l_h = 0.f;          // this warp's share of the row sum, relative to m_ref
+  bool failed = false;      // warp-uniform
 
-  for (int j = 0; j < pr.n; ++j) {
-    const uint32_t it = ps.kv + j, b = it & 1;
-    const int tile0 = (pr.t0 + j) * kKVTile;
+  for (int t = hf; t < n; t += 2) {
+    const uint32_t it = ps.kv + t, b = it & 1;
+    const int tile0 = (pr.t0 + t) * kKVTile;
     const bool masked_tile = tile0 + kKVTile - 1 > mask_from;  // uniform over the CTA
-    float s[64];
-    float mx = -INFINITY;
-    if (!failed) failed = !pwait_warp(bars + (L::B_SF + b) * 8, (it >> 1) & 1, P, pa);
-    if (!failed) {
-      tc_fence_after();
-      uint32_t r0[32], r1[32];
-      tmem_ld32x2(tmem + lane_base + L::T_S + 128 * b + 64 * hf, r0, r1);
+    // Straight-line body: once the CTA has aborted every wait returns at once
+    // and the tensor-memory work below only moves stale values, whose results
+    // are never stored (`failed`).
+    failed |= !pwait_warp(bars + (L::B_SF + b) * 8, (it >> 1) & 1, P, pa);
+    tc_fence_after();
+    float s[128];
+    {
+      uint32_t r[128];
+      tmem_ld128(tmem + lane_base + L::T_S + 128 * b, r);
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        s[c] = __uint_as_float(r0[c]);
-        s[32 + c] = __uint_as_float(r1[c]);
-      }
-      // S_b may be overwritten once every softmax warp of both CTAs has it
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) handoff_arrive(lbars + (L::B_SE + b) * 8);
-      if (masked_tile) {
-        const int k0 = tile0 + 64 * hf;
-#pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (k0 + c > lim) s[c] = -INFINITY;
-      }
-      float a[22];  // 64 -> 22 -> 8 -> 3 -> 1 with three-input max
-#pragma unroll
-      for (int c = 0; c < 21; ++c) a[c] = max3(s[3 * c], s[3 * c + 1], s[3 * c + 2]);
-      a[21] = s[63];
-      float bb[8];
-#pragma unroll
-      for (int c = 0; c < 7; ++c) bb[c] = max3(a[3 * c], a[3 * c + 1], a[3 * c + 2]);
-      bb[7] = a[21];
-      mx = fmaxf(max3(bb[0], bb[1], bb[2]), max3(max3(bb[3], bb[4], bb[5]), bb[6], bb[7]));
+      for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(r[c]);
     }
-    // the two column halves of each row meet (double-buffered by tile parity:
-    // a half writes the slot of tile it + 2 only after both passed tile it + 1)
-    xmax[((it & 1) * 2 + hf) * kQTile + row] = mx;
-    named_bar_sync(pair_bar, 64);
-    mx = fmaxf(mx, xmax[((it & 1) * 2 + (hf ^ 1)) * kQTile + row]);
-    if (failed) continue;
+    // S_b may be overwritten once all its readers in both CTAs have it
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) handoff_arrive(lbars + (L::B_SE + b) * 8);
+    if (masked_tile) {
+#pragma unroll
+      for (int c = 0; c < 128; ++c)
+        if (tile0 + c > lim) s[c] = -INFINITY;
+    }
+    // row max: eight chains of three-input max (few live temporaries beside s)
+    float mc[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) mc[k] = fmaxf(s[k], s[8 + k]);
+#pragma unroll
+    for (int c = 16; c < 128; c += 16)
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mc[k] = max3(mc[k], s[c + k], s[c + 8 + k]);
+    float mx = fmaxf(max3(mc[0], mc[1], mc[2]), max3(max3(mc[3], mc[4], mc[5]), mc[6], mc[7]));
+    // the reference after tile t - 1, from its owner (none before the unit's first tile)
+    if (t >= 1) {
+      named_bar_sync(hand_from, 64);
+      const float m_prev = xref[(hf ^ 1) * kQTile + row];
+      if (m_prev > m_ref) {  // monotone: rescale this warp's share to the newer reference
+        l_h = (m_ref == -INFINITY) ? 0.f : l_h * ex2(m_ref - m_prev);
+        m_ref = m_prev;
+      }
+    }
+    // Lazy rescaling: the reference is raised only when the row max exceeds it
+    // by more than 8 (log2 units), so every weight is <= 2^8.
     mx *= sc;
-    // Lazy rescaling: the reference max is raised only when the row max
-    // exceeds it by more than 8 (log2 units), so every weight is <= 2^8. Both
-    // halves of a row see the same maxima, so they take the same decisions.
     float alpha = 1.f;
     bool rescale = false;
-    if (mx > m_run + 8.f) {
-      alpha = ex2(m_run - mx);         // 0 on the unit's first tile
-      rescale = (m_run != -INFINITY);  // O holds earlier tiles' sums
-      m_run = mx;
+    if (mx > m_ref + 8.f) {
+      alpha = ex2(m_ref - mx);         // 0 when nothing was seen yet
+      rescale = (m_ref != -INFINITY);  // O holds earlier tiles' sums
+      l_h *= alpha;
+      m_ref = mx;
     }
-    const float m_use = (m_run == -INFINITY) ? 0.f : m_run;  // fully masked row so far
+    // hand the reference on to the owner of tile t + 1 before the exponentials
+    if (t + 1 < n) {
+      xref[hf * kQTile + row] = m_ref;
+      asm volatile("bar.arrive %0, 64;" ::"r"(hand_to) : "memory");
+    }
+    const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;  // fully masked row so far
+    // P_b is free once P_{it-2} V has completed
+    if (it >= 2) failed |= !pwait_warp(bars + (L::B_PE + b) * 8, ((it - 2) >> 1) & 1, P, pa);
+    tc_fence_after();
+    // P = 2^(s sc - m) as bf16 pairs over P_b, one 64-key half at a time (each
+    // half stored as soon as it is packed), and the row sum of the unrounded
+    // weights
+    const uint64_t sc2 = f2_pack(sc, sc), nm2 = f2_pack(-m_use, -m_use);
+    uint64_t acc[4];
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      uint32_t pk[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        const int k = 64 * hh + 2 * c;
+        float x0, x1;
+        f2_unpack(ffma2(f2_pack(s[k], s[k + 1]), sc2, nm2), x0, x1);
+        const float p0 = ex2(x0), p1 = ex2(x1);
+        const uint64_t p2 = f2_pack(p0, p1);
+        pk[c] = pair_pack(p0, p1);
+        acc[c & 3] = (hh == 0 && c < 4) ? p2 : fadd2(acc[c & 3], p2);
+      }
+      if (hh == 0)
+        tmem_st32_nowait(tmem + lane_base + L::T_P + 64 * b, pk);
+      else
+        tmem_st32(tmem + lane_base + L::T_P + 64 * b + 32, pk);  // waits for both stores
+    }
+    {
+      float a0, a1;
+      f2_unpack(fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3])), a0, a1);
+      l_h += a0 + a1;
+    }
+    // O to the raised reference, after P_{it-1} V and before this tile's P V
+    // (issued only after the P-ready arrival below); a rescale never happens
+    // on a unit's first tile, so it - 1 belongs to this unit
     if (__any_sync(0xffffffffu, rescale)) {
-      // O must include P_{it-1} V first (a rescale never happens on a unit's
-      // first tile, so it - 1 belongs to this unit)
-      failed = !pwait_warp(bars + (L::B_PE + ((it - 1) & 1)) * 8, ((it - 1) >> 1) & 1, P, pa);
-      if (failed) continue;
+      failed |= !pwait_warp(bars + (L::B_PE + ((it - 1) & 1)) * 8, ((it - 1) >> 1) & 1, P, pa);
       tc_fence_after();
       const float f = rescale ? alpha : 1.f;
 #pragma unroll
-      for (int cb = 0; cb < 2; ++cb) {
+      for (int cb = 0; cb < D / 32; ++cb) {
         uint32_t ov[32];
-        const uint32_t oc = tmem + lane_base + L::T_O + 64 * hf + 32 * cb;
+        const uint32_t oc = tmem + lane_base + L::T_O + 32 * cb;
         tmem_ld32(oc, ov);
 #pragma unroll
         for (int q = 0; q < 32; ++q) ov[q] = __float_as_uint(__uint_as_float(ov[q]) * f);
         tmem_st32(oc, ov);
       }
     }
-    // P = 2^(s sc - m) as bf16 pairs, and this half's row sum of the
-    // unrounded weights
-    const uint64_t sc2 = f2_pack(sc, sc), nm2 = f2_pack(-m_use, -m_use);
-    uint32_t pk[32];
-    uint64_t acc[4];
-#pragma unroll
-    for (int c = 0; c < 32; ++c) {
-      float x0, x1;
-      f2_unpack(ffma2(f2_pack(s[2 * c], s[2 * c + 1]), sc2, nm2), x0, x1);
-      float p0, p1;
-      uint64_t p2;
-      if (!masked_tile && (c & 7) >= 8 - kPairPolyPairs) {
-        p2 = exp2_poly2(x0, x1);
-        f2_unpack(p2, p0, p1);
-      } else {
-        p0 = ex2(x0);
-        p1 = ex2(x1);
-        p2 = f2_pack(p0, p1);
-      }
-      pk[c] = pair_pack(p0, p1);
-      acc[c & 3] = (c < 4) ? p2 : fadd2(acc[c & 3], p2);
-    }
-    float lt;
-    {
-      float a0, a1;
-      f2_unpack(fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3])), a0, a1);
-      lt = a0 + a1;
-    }
-    l_run = l_run * alpha + lt;
-    // P_b is free once P_{it-2} V has completed
-    if (it >= 2) {
-      failed = !pwait_warp(bars + (L::B_PE + b) * 8, ((it - 2) >> 1) & 1, P, pa);
-      if (failed) continue;
-      tc_fence_after();
-    }
-    tmem_st32(tmem + lane_base + L::T_P + 64 * b + 32 * hf, pk);  // waits for the store
     tc_fence_before();
     __syncwarp();
     if (lane == 0) handoff_arrive(lbars + (L::B_PF + b) * 8);
@@ -515,10 +540,17 @@ POD_DEV bool pair_softmax(const Plan& P, const PrefillRange& pr, int rank, uint8
   }
   ps.kv += pr.n;
   ps.units++;
-  // the row sum of both halves
-  xsum[hf * kQTile + row] = l_run;
-  named_bar_sync(pair_bar, 64);
-  const float l_tot = l_run + xsum[(hf ^ 1) * kQTile + row];
+  // The two warps' references and row-sum shares meet: the larger reference
+  // is the final one (references only grow), and each share is rescaled to it.
+  xfin[hf * kQTile + row] = m_ref;
+  xfin[(2 + hf) * kQTile + row] = l_h;
+  named_bar_sync(kBarFinal0 + q4, 64);
+  const float m_o = xfin[(hf ^ 1) * kQTile + row], l_o = xfin[(2 + (hf ^ 1)) * kQTile + row];
+  const float m_run = fmaxf(m_ref, m_o);
+  const float l_tot = (m_run == -INFINITY)
+                          ? 0.f
+                          : ((m_ref == -INFINITY) ? 0.f : l_h * ex2(m_ref - m_run)) +
+                                ((m_o == -INFINITY) ? 0.f : l_o * ex2(m_o - m_run));
   const bool valid = tile_ok && (q_local < R.chunk) && !failed;
   const size_t out_row = (size_t)(R.q_row0 + q_local);
   const float lse2 = (l_tot > 0.f) ? (m_run + log2f(l_tot)) : -INFINITY;
@@ -569,13 +601,13 @@ POD_DEV bool pair_softmax(const Plan& P, const PrefillRange& pr, int rank, uint8
   }
   if (valid && hf == 0) P.ppart_lse[(size_t)(slot0 + pr.split) * kQTile + row] = lse2 * kLn2;
   __threadfence();
-  named_bar_sync(6, kSoftmaxWarps * 32);
+  named_bar_sync(kBarSoftmaxAll, kSoftmaxWarps * 32);
   if (tid == 0) {
     // a missing tile has no group; after a failure nobody merges
     const int old = (*pa.flag || !tile_ok) ? -1 : atomicAdd(P.pgroup_ctr + pr.group[rank], 1);
     *merge_flag = (old == pr.n_split - 1);
   }
-  named_bar_sync(6, kSoftmaxWarps * 32);
+  named_bar_sync(kBarSoftmaxAll, kSoftmaxWarps * 32);
   if (*merge_flag && !failed && valid) {
     // The last split to finish merges all of them in split order (each
     // thread: one row, its 64 columns): O = sum_s w_s O_s / sum_s w_s,
