@@ -523,10 +523,13 @@ def run_sweep(args, rank, world, local):
             [0, 4, 8, 12, 16, 20, 24, 28, 29, 30, 31]
         workloads = ["chunked16k_%d" % i for i in points]
         variants = SWEEP_VARIANTS
-    else:  # policies on the full-size configurations
+    else:  # policies on the full-size configurations, with either prefill tile
         workloads = args.sweep_points.split(",") if args.sweep_points else \
             ["llama3_8b", "decode_heavy", "long_context", "paged"]
-        variants = SWEEP_POLICIES
+        variants = {}
+        for tile, tenv in (("pair", {}), ("1sm", {"POD_ATTN_PREFILL_TILE": "1sm"})):
+            for pname, penv in SWEEP_POLICIES.items():
+                variants["%s_%s" % (tile, pname)] = dict(tenv, **penv)
     for name in workloads:
         batch = W.make_batch(W.get_config(name))
         db = pa.DeviceBatch(batch, device=dev)

@@ -123,8 +123,7 @@ struct FusedLayout {
   static constexpr int B_SE = B_SF + 2;                 // S_i free (its P read by PV_i) [2]
   static constexpr int B_PF = B_SE + 2;                 // P_i in TMEM, one arrival per warp [2]
   static constexpr int B_OR = B_PF + 2;                 // O_i final for the unit [2]
-  static constexpr int B_DEC = B_OR + 2;
-  static constexpr int N_BARS = B_DEC + kFusedWarps * kFusedDecStages;  // a ring per warp
+  static constexpr int N_BARS = B_OR + 2;
   static constexpr int MISC_OFF = BAR_OFF + N_BARS * 8;
   static constexpr int TOTAL = MISC_OFF + 64;
   static_assert(TOTAL <= 227 * 1024, "fused CTA exceeds the shared memory of an SM");
@@ -140,8 +139,8 @@ struct DecodeLayout {
   static constexpr int ROW = D * 2 + 16;
   static constexpr int STAGE = 2 * kDecTile * ROW;
   static constexpr int WARP = kDecodeStages * STAGE;
-  static constexpr int BAR_OFF = kDecodeWarps * WARP;
-  static constexpr int SMEM_BYTES = BAR_OFF + kDecodeWarps * kDecodeStages * 8 + 16;
+  static constexpr int FLAG_OFF = kDecodeWarps * WARP;  // one abort flag per warp
+  static constexpr int SMEM_BYTES = FLAG_OFF + kDecodeWarps * 4;
 };
 
 // ============================================================= LSE merge
@@ -258,15 +257,27 @@ POD_DEV void merge_decode_group(const Plan& P, const DecodeReq& R, int r, int g,
 
 // ============================================================= decode unit
 // One warp, one unit (request r, KV head g, keys [kbeg, kend)). The ring of
-// `NST` stages lives at `wsm` (each stage: 16 K rows then 16 V rows, padded);
-// `bar0` is the shared address of NST mbarriers. `ring` counts tiles this warp
-// has staged so far (carries the mbarrier phases across units).
+// `NST` stages lives at `wsm` (each stage: 16 K rows then 16 V rows, padded).
+// `ring` counts tiles this warp has staged so far (the stage slot rotates
+// across units).
+//
+// Staging: every lane copies 16-byte pieces with cp.async (one commit group
+// per stage), so a warp instruction moves two whole 256-byte rows (d = 128)
+// and a stage takes D / 8 instructions per lane. A row of one KV head is the
+// only contiguous run of a (token, head)-major cache, and 256-byte bulk
+// (TMA) copies, one per lane, took far longer to issue than the stage's
+// arithmetic; plain asynchronous copies issue at the load/store rate and need
+// no mbarrier and no proxy fence between a stage's reads and its refill.
 template <int D, int NST>
-POD_DEV bool decode_unit_warp(const Plan& P, int u, uint8_t* wsm, uint32_t bar0, uint32_t& ring,
-                              int lane, bool inline_merge, volatile int* abort_flag) {
+POD_DEV bool decode_unit_warp(const Plan& P, int u, uint8_t* wsm, uint32_t& ring, int lane,
+                              bool inline_merge, volatile int* abort_flag) {
+  static_assert(NST >= 1 && NST <= 8, "cp.async.wait_group counts at most 7 pending groups");
   constexpr int ROW = D * 2 + 16;
   constexpr int STAGE = 2 * kDecTile * ROW;
   constexpr int KS = D / 16;
+  constexpr int CH = D * 2 / 16;  // 16-byte pieces per row
+  constexpr int RPI = 32 / CH;    // rows per warp instruction
+  static_assert(2 * kDecTile % RPI == 0, "a stage is a whole number of warp instructions");
   const int r = P.dunit_req[u];
   const DecodeReq R = P.dreq[r];
   const int Hk = P.Hk, G = P.G;
@@ -295,40 +306,46 @@ POD_DEV bool decode_unit_warp(const Plan& P, int u, uint8_t* wsm, uint32_t bar0,
     }
   }
   const size_t row_elems = (size_t)Hk * D;
-  auto row_off = [&](int key) -> size_t {
-    if (P.paged) {
-      int phys = __ldg(P.bt_d + (size_t)R.bt_row * P.bt_stride_d + (key >> 4));
-      phys = min(max(phys, 0), P.pool_blocks - 1);  // never read outside the pool
-      return ((size_t)phys * 16 + (key & 15)) * row_elems + (size_t)g * D;
-    }
-    return (size_t)key * row_elems + (size_t)g * D;
-  };
   const uint16_t* kbase = P.paged ? P.k_pool : R.k;
   const uint16_t* vbase = P.paged ? P.v_pool : R.v;
   const uint32_t wsm_a = smem_u32(wsm);
 #if POD_L2_HINTS
   const uint64_t once = l2_evict_first();  // decode K/V is read once
 #endif
+  const int col = lane % CH, rsub = lane / CH;  // this lane's piece and row phase
 
+  // Stage t: keys kbeg + 16 t .. +15 (a ragged tail re-reads the last valid
+  // row; those keys are masked below). Split lengths are multiples of 16, so
+  // a stage never crosses a 16-token page: one block-table entry per stage.
   auto issue = [&](int t) {
-    const uint32_t it = ring + t;
-    const uint32_t st = it % NST;
-    const uint32_t bar = bar0 + st * 8;
-    if (lane == 0) mbar_expect_tx(bar, 2 * kDecTile * D * 2);
-    __syncwarp();
-    int key = kbeg + t * kDecTile + (lane & 15);
-    key = min(key, kend - 1);  // ragged tail: re-read a valid row, masked below
-    const size_t off = row_off(key);
-    const uint16_t* src = (lane < 16) ? (kbase + off) : (vbase + off);
-    const uint32_t dst = wsm_a + st * STAGE + (lane < 16 ? 0 : kDecTile * ROW) + (lane & 15) * ROW;
+    const uint32_t st = (ring + t) % NST;
+    const int key0 = kbeg + t * kDecTile;
+    size_t base_off;
+    if (P.paged) {
+      int phys = __ldg(P.bt_d + (size_t)R.bt_row * P.bt_stride_d + (key0 >> 4));
+      phys = min(max(phys, 0), P.pool_blocks - 1);  // never read outside the pool
+      base_off = (size_t)phys * kDecTile * row_elems + (size_t)g * D;
+    } else {
+      base_off = (size_t)key0 * row_elems + (size_t)g * D;
+    }
+    const int last = kend - 1 - key0;  // last valid key of the stage, 0..15
+    const uint32_t dst0 = wsm_a + st * STAGE + col * 16;
+#pragma unroll
+    for (int i = 0; i < 2 * kDecTile / RPI; ++i) {
+      const int row = i * RPI + rsub;  // 0..15 K rows, 16..31 V rows
+      const int k = min(row & (kDecTile - 1), last);
+      const uint16_t* src = (row < kDecTile ? kbase : vbase) + base_off + (size_t)k * row_elems +
+                            col * 8;
+      const uint32_t dst = dst0 + (row < kDecTile ? 0 : kDecTile * ROW) + (row & (kDecTile - 1)) * ROW;
 #if POD_L2_HINTS
-    bulk_load_hint(dst, src, D * 2, bar, once);
+      cp_async16_hint(dst, src, once);
 #else
-    bulk_load(dst, src, D * 2, bar);
+      cp_async16(dst, src);
 #endif
+    }
+    cp_async_commit();
   };
 
-  fence_proxy_async_smem();
   int issued = min(NST, n_tiles);  // tiles [0, issued) have been issued
   for (int t = 0; t < issued; ++t) issue(t);
 
@@ -340,9 +357,11 @@ POD_DEV bool decode_unit_warp(const Plan& P, int u, uint8_t* wsm, uint32_t bar0,
   bool ok = true;
 
   for (int t = 0; t < n_tiles; ++t) {
-    const uint32_t it = ring + t;
-    const uint32_t st = it % NST;
-    if (!wait_bar_warp(bar0 + st * 8, (it / NST) & 1, P, abort_flag)) {
+    const uint32_t st = (ring + t) % NST;
+    // stage t landed: the groups issued after it may still be in flight
+    cp_async_wait_pending(issued - 1 - t);
+    __syncwarp();  // every lane's pieces visible to the whole warp
+    if (__any_sync(0xffffffffu, *abort_flag != 0)) {
       ok = false;
       break;
     }
@@ -400,24 +419,19 @@ POD_DEV bool decode_unit_warp(const Plan& P, int u, uint8_t* wsm, uint32_t bar0,
                 a);
       mma_16816(o[mt], a, b0, b1);
     }
-    __syncwarp();
+    __syncwarp();  // every lane's reads of this stage are done before its refill
     if (t + NST < n_tiles) {
-      fence_proxy_async_smem();
       issue(t + NST);
       issued = t + NST + 1;
     }
   }
-  if (!ok) {
-    // Abort: wait (bounded) for the copies this warp still has in flight --
-    // the last NST issued tiles -- so no copy lands after the CTA exits.
-    for (int t = max(0, issued - NST); t < issued; ++t) {
-      const uint32_t it = ring + t;
-      drain_bar(bar0 + (it % NST) * 8, (it / NST) & 1, P.wait_budget);
-    }
-    ring += n_tiles;
-    return false;
-  }
+  // All copies landed (on an abort too, so none lands after the CTA exits).
+  // The ring may next hold a prefill tile written by TMA: order this warp's
+  // generic-proxy accesses before any later async-proxy write.
+  cp_async_wait_pending(0);
+  fence_proxy_async_smem();
   ring += n_tiles;
+  if (!ok) return false;
 
   // l: sum of lane partials over the 8 lanes sharing q4.
 #pragma unroll
@@ -623,9 +637,8 @@ __global__ void __launch_bounds__(kFusedThreads, kFusedSlotsPerSm)
             if (lane == 0) misc[6] = 1;
             break;
           }
-          if (!decode_unit_warp<D, kFusedDecStages>(P, u, sm + warp * L::DEC_WARP,
-                                                    bars + (L::B_DEC + warp * kFusedDecStages) * 8,
-                                                    dec_ring, lane, true, abort_flag))
+          if (!decode_unit_warp<D, kFusedDecStages>(P, u, sm + warp * L::DEC_WARP, dec_ring, lane,
+                                                    true, abort_flag))
             break;
         }
       }
@@ -646,7 +659,6 @@ __global__ void __launch_bounds__(kFusedThreads, kFusedSlotsPerSm)
         break;
       }
       if (!decode_unit_warp<D, kFusedDecStages>(P, u, sm + L::SIDE_OFF + sw * L::DEC_WARP,
-                                                bars + (L::B_DEC + warp * kFusedDecStages) * 8,
                                                 side_ring, lane, true, abort_flag))
         break;
     }
@@ -823,9 +835,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             if (lane == 0) misc[kMiscDEmpty] = 1;
             break;
           }
-          if (!decode_unit_warp<D, L::ROLE_DEC_ST>(P, u, sm + warp * L::ROLE_DEC_WARP,
-                                                  bars + (L::B_DEC + warp * L::ROLE_DEC_ST) * 8,
-                                                  dec_ring, lane, true, abort_flag))
+          if (!decode_unit_warp<D, L::ROLE_DEC_ST>(P, u, sm + warp * L::ROLE_DEC_WARP, dec_ring,
+                                                  lane, true, abort_flag))
             break;
         }
       }
@@ -845,10 +856,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         if (lane == 0) misc[kMiscDEmpty] = 1;
         break;
       }
-      if (!decode_unit_warp<D, L::SIDE_DEC_ST>(
-              P, u, sm + L::SIDE_OFF + sw * L::SIDE_DEC_WARP,
-              bars + (L::B_DEC + L::TURN_WARPS * L::ROLE_DEC_ST + sw * L::SIDE_DEC_ST) * 8, side_ring,
-              lane, true, abort_flag))
+      if (!decode_unit_warp<D, L::SIDE_DEC_ST>(P, u, sm + L::SIDE_OFF + sw * L::SIDE_DEC_WARP,
+                                               side_ring, lane, true, abort_flag))
         break;
     }
   }
@@ -897,15 +906,8 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = smem_raw;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t bar0 = smem_u32(sm + L::BAR_OFF) + warp * kDecodeStages * 8;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::BAR_OFF +
-                                                              kDecodeWarps * kDecodeStages * 8) +
-                             warp;
-  if (lane == 0) {
-    for (int i = 0; i < kDecodeStages; ++i) mbar_init(bar0 + i * 8, 1);
-    fence_mbar_init();
-    *abort_flag = 0;
-  }
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::FLAG_OFF) + warp;
+  if (lane == 0) *abort_flag = 0;
   __syncwarp();
   uint32_t ring = 0;
   while (true) {
@@ -913,7 +915,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
     if (lane == 0) u = atomicAdd(P.ctl + 1, 1);
     u = __shfl_sync(0xffffffffu, u, 0);
     if (u >= P.n_decode_units) break;
-    if (!decode_unit_warp<D, kDecodeStages>(P, u, sm + warp * L::WARP, bar0, ring, lane, false,
+    if (!decode_unit_warp<D, kDecodeStages>(P, u, sm + warp * L::WARP, ring, lane, false,
                                             abort_flag))
       break;
   }

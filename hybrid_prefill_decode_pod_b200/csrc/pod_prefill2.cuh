@@ -79,8 +79,7 @@ struct PairLayout {
   static constexpr int B_OR = B_PE + 2;           // O final for the unit
   static constexpr int B_MB = B_OR + 1;           // peer: the leader posted a claim
   static constexpr int B_ACK = B_MB + 1;          // leader: the peer read the claim
-  static constexpr int B_DEC = B_ACK + 1;         // decode rings: role warps, then side warps
-  static constexpr int N_BARS = B_DEC + TURN_WARPS * ROLE_DEC_ST + kSideDecWarps * SIDE_DEC_ST;
+  static constexpr int N_BARS = B_ACK + 1;
   static constexpr int MISC_OFF = BAR_OFF + N_BARS * 8;
   static constexpr int TOTAL = MISC_OFF + 64;
   static_assert(TOTAL <= 227 * 1024, "pair CTA exceeds the shared memory of an SM");
