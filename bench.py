@@ -488,9 +488,10 @@ def run_gpu(args, rank, world, local):
 # §5.4.1: the prefill tile's size). Each is a set of planner levers read when
 # a context is created.
 SWEEP_VARIANTS = {
-    "pair_model": {},                                        # CTA-pair tile, split model
-    "pair_nosplit": {"POD_ATTN_PREFILL_SPLIT": "1"},
-    "pair_uncapped8": {"POD_ATTN_PREFILL_SPLIT": "-8"},      # 8 splits, two-wave cap off
+    "pair_model": {"POD_ATTN_PREFILL_TILE": "pair"},         # CTA-pair tile, split model
+    "pair_nosplit": {"POD_ATTN_PREFILL_TILE": "pair", "POD_ATTN_PREFILL_SPLIT": "1"},
+    "pair_uncapped8": {"POD_ATTN_PREFILL_TILE": "pair",      # 8 splits, two-wave cap off
+                       "POD_ATTN_PREFILL_SPLIT": "-8"},
     "1sm_model": {"POD_ATTN_PREFILL_TILE": "1sm"},           # one-SM pair tile, split model
     "1sm_uncapped8": {"POD_ATTN_PREFILL_TILE": "1sm", "POD_ATTN_PREFILL_SPLIT": "-8"},
 }
@@ -527,7 +528,8 @@ def run_sweep(args, rank, world, local):
         workloads = args.sweep_points.split(",") if args.sweep_points else \
             ["llama3_8b", "decode_heavy", "long_context", "paged"]
         variants = {}
-        for tile, tenv in (("pair", {}), ("1sm", {"POD_ATTN_PREFILL_TILE": "1sm"})):
+        for tile, tenv in (("1sm", {"POD_ATTN_PREFILL_TILE": "1sm"}),
+                           ("pair", {"POD_ATTN_PREFILL_TILE": "pair"})):
             for pname, penv in SWEEP_POLICIES.items():
                 variants["%s_%s" % (tile, pname)] = dict(tenv, **penv)
     for name in workloads:

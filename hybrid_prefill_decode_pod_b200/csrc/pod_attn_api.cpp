@@ -785,11 +785,14 @@ int pod_attn_create(pod_attn_ctx** out, const pod_attn_config* cfg) {
   }
   if (const char* e = std::getenv("POD_ATTN_DEC_SPLIT"))
     c->dec_split = std::max(0, std::atoi(e)) / kDecTile * kDecTile;
-  // The CTA-pair prefill tile (head_dim 128) unless switched off; its
+  // The one-SM prefill tile serves every head_dim by default: it measured
+  // faster than the CTA-pair tile on every hybrid workload of the benchmark
+  // (the pair's single MMA-issuing thread sets its pace). The pair tile
+  // (head_dim 128) is selected with POD_ATTN_PREFILL_TILE=pair; its
   // persistent launch uses every cluster of two that fits at once.
   if (D == 128) {
     const char* e = std::getenv("POD_ATTN_PREFILL_TILE");
-    if (!(e && !std::strcmp(e, "1sm"))) {
+    if (e && !std::strcmp(e, "pair")) {
       int clusters = 0;
       if (pair_max_clusters(&clusters) != cudaSuccess) return fail(POD_ECUDA);
       if (clusters >= 1) {
