@@ -199,7 +199,8 @@ POD_DEV void merge_rows_warp(const float* po, long long po_split, long long po_r
       W[rb] += w[rb];
     }
     const int cnt = min(32, n - s0);
-#pragma unroll 2
+    // loads of several splits in flight: the merge is L2-latency bound
+#pragma unroll(RB == 1 ? 8 : 2)
     for (int t = 0; t < cnt; ++t) {
       const float* src = po + (long long)(s0 + t) * po_split + lane * PER;
       float x[RB][PER];
@@ -921,25 +922,34 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
   }
 }
 
-// One warp per (decode request, KV head) group whose KV range was split.
+// One warp per decode query row (request r, query head h) whose KV range was
+// split: its KV head's partials are merged for that row alone, so the launch
+// has H x requests warps in flight instead of Hk x requests. The per-row
+// arithmetic is that of the fused kernel's last-arriver merge (which merges
+// all G rows of a group in one warp), so both give the same bits.
 // With kFlagPoisonOnStatus set, a non-zero status word (a decode warp gave up
-// on a bounded wait) makes every group write NaN instead, so a call whose
+// on a bounded wait) makes every row write NaN instead, so a call whose
 // partial results are incomplete cannot be mistaken for a result.
 template <int D>
 __global__ void __launch_bounds__(128) pod_merge_kernel(const __grid_constant__ Plan P) {
   const int gw = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (gw >= P.n_decode_reqs * P.Hk) return;
-  const int r = gw / P.Hk, g = gw - (gw / P.Hk) * P.Hk;
+  if (gw >= P.n_decode_reqs * P.H) return;
+  const int r = gw / P.H, h = gw - r * P.H;
+  const int g = h / P.G, i = h - g * P.G;
   if ((P.flags & kFlagPoisonOnStatus) && *reinterpret_cast<volatile const int*>(P.status) != 0) {
-    uint16_t* o = P.o_d + ((size_t)r * P.H + (size_t)g * P.G) * D;
-    for (int i = lane; i < P.G * D; i += 32) o[i] = 0x7FC0u;  // bf16 quiet NaN
-    if (lane < P.G) P.lse_d[(size_t)r * P.H + (size_t)g * P.G + lane] = __int_as_float(0x7FC00000);
+    uint16_t* o = P.o_d + ((size_t)r * P.H + h) * D;
+    for (int k = lane; k < D; k += 32) o[k] = 0x7FC0u;  // bf16 quiet NaN
+    if (lane == 0) P.lse_d[(size_t)r * P.H + h] = __int_as_float(0x7FC00000);
     return;
   }
   const DecodeReq R = P.dreq[r];
   if (R.n_split <= 1) return;
-  merge_decode_group<D>(P, R, r, g, lane);
+  const int slot0 = R.slot0 + g;
+  merge_rows_warp<D, 1>(P.dpart_o + (size_t)slot0 * kMaxGroup * D, (long long)P.Hk * kMaxGroup * D,
+                        D, P.dpart_lse + (size_t)slot0 * kMaxGroup, (long long)P.Hk * kMaxGroup, 1,
+                        R.n_split, i, P.G, P.o_d + ((size_t)r * P.H + (size_t)g * P.G) * D, D,
+                        P.lse_d + (size_t)r * P.H + (size_t)g * P.G, 1, lane);
 }
 
 // ============================================================= host-side launchers
@@ -1035,7 +1045,7 @@ cudaError_t launch_decode(const Plan& P, int max_grid, cudaStream_t s) {
 }
 
 cudaError_t launch_merge(const Plan& P, cudaStream_t s) {
-  const int rows = P.n_decode_reqs * P.Hk;
+  const int rows = P.n_decode_reqs * P.H;  // one warp per query row, four per block
   const int grid = (rows + 3) / 4;
   if (grid == 0) return cudaSuccess;
   if (P.D == 128)
