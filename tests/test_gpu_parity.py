@@ -109,6 +109,30 @@ def test_pair_and_one_sm_prefill_tiles_match_oracle(shape):
             compare(ref, out)
 
 
+POLICIES = ["front", "prefill_first", "even", "proportional", "balanced", "decode_first"]
+
+
+@pytest.mark.parametrize("tile", ["1sm", "pair"])
+def test_every_role_policy_matches_oracle_and_agrees_bitwise(tile):
+    """The role policy decides which SM runs which unit and when, never what a
+    unit computes: every policy gives the same bits on the same plan, and
+    they match the oracle."""
+    b = W.make_custom(8, 2, 128, [(1500, 400), (0, 130)], [64, 700, 3000, 9000, 17], seed=23)
+    ref = oracle.hybrid(b)
+    first = None
+    for policy in POLICIES:
+        with plan_env(POD_ATTN_PREFILL_TILE=tile, POD_ATTN_POLICY=policy):
+            out, plan = run(b, "fused")
+        assert (plan["pair_clusters"] > 0) == (tile == "pair")
+        compare(ref, out)
+        if first is None:
+            first = (out, plan)
+        else:
+            assert plan["prefill_split"] == first[1]["prefill_split"]
+            assert plan["decode_split_len"] == first[1]["decode_split_len"]
+            assert bitwise_equal(first[0], out), policy
+
+
 def test_prefill_only_and_decode_only_match_hybrid():
     b = W.make_custom(8, 2, 128, [(700, 300)], [3000, 20], seed=17)
     h, _ = run(b, "fused")
@@ -259,7 +283,9 @@ FULL_SIZE = [("llama3_8b", "fused"), ("decode_heavy", "fused"),
              ("llama2_7b_mha", "fused"), ("yi6b_g8", "fused"), ("d64_mix", "fused"),
              ("many_chunks", "fused"), ("many_chunks", "serial"),
              # a late chunk of the chunked 16K prompt (prior 15872 + 512, 64 decodes)
-             ("chunked16k_31", "fused")]
+             ("chunked16k_31", "fused"),
+             # the CTA-pair prefill tile (POD_ATTN_PREFILL_TILE=pair)
+             ("long_context", "fused+pair"), ("paged", "fused+pair")]
 
 
 @pytest.mark.slow
@@ -269,5 +295,8 @@ def test_full_size_configs_every_element(name, mode):
     every output element against the fp64 oracle. SERIAL and TWO_STREAM take
     their own prefill plans (they may split the KV range where FUSED does not)."""
     b, ref = _full_ref(name)
-    out, plan = run(b, mode)
+    mode, _, tile = mode.partition("+")
+    with plan_env(POD_ATTN_PREFILL_TILE=tile or "1sm"):
+        out, plan = run(b, mode)
+    assert (plan["pair_clusters"] > 0) == (tile == "pair")
     compare(ref, out)
