@@ -330,20 +330,33 @@ POD_DEV bool decode_unit_warp(const Plan& P, int u, uint8_t* wsm, uint32_t& ring
       base_off = (size_t)key0 * row_elems + (size_t)g * D;
     }
     const int last = kend - 1 - key0;  // last valid key of the stage, 0..15
-    const uint32_t dst0 = wsm_a + st * STAGE + col * 16;
-#pragma unroll
-    for (int i = 0; i < 2 * kDecTile / RPI; ++i) {
-      const int row = i * RPI + rsub;  // 0..15 K rows, 16..31 V rows
-      const int k = min(row & (kDecTile - 1), last);
-      const uint16_t* src = (row < kDecTile ? kbase : vbase) + base_off + (size_t)k * row_elems +
-                            col * 8;
-      const uint32_t dst = dst0 + (row < kDecTile ? 0 : kDecTile * ROW) + (row & (kDecTile - 1)) * ROW;
+    // this lane's piece of key rows rsub, rsub + RPI, ... of K (then V)
+    const uint32_t dk = wsm_a + st * STAGE + rsub * ROW + col * 16;
+    const uint16_t* sk = kbase + base_off + col * 8;
+    const uint16_t* sv = vbase + base_off + col * 8;
 #if POD_L2_HINTS
-      cp_async16_hint(dst, src, once);
+#define POD_DEC_COPY(d, s) cp_async16_hint(d, s, once)
 #else
-      cp_async16(dst, src);
+#define POD_DEC_COPY(d, s) cp_async16(d, s)
 #endif
+    if (last >= kDecTile - 1) {  // a full stage: rows advance by RPI rows of the cache
+      const size_t step = (size_t)RPI * row_elems;
+      sk += (size_t)rsub * row_elems;
+      sv += (size_t)rsub * row_elems;
+#pragma unroll
+      for (int i = 0; i < kDecTile / RPI; ++i, sk += step, sv += step) {
+        POD_DEC_COPY(dk + i * RPI * ROW, sk);
+        POD_DEC_COPY(dk + (kDecTile + i * RPI) * ROW, sv);
+      }
+    } else {  // the ragged tail re-reads the last valid row (masked in the softmax)
+#pragma unroll
+      for (int i = 0; i < kDecTile / RPI; ++i) {
+        const size_t k = (size_t)min(i * RPI + rsub, last) * row_elems;
+        POD_DEC_COPY(dk + i * RPI * ROW, sk + k);
+        POD_DEC_COPY(dk + (kDecTile + i * RPI) * ROW, sv + k);
+      }
     }
+#undef POD_DEC_COPY
     cp_async_commit();
   };
 
@@ -392,24 +405,38 @@ POD_DEV bool decode_unit_warp(const Plan& P, int u, uint8_t* wsm, uint32_t& ring
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
     }
-    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);  // finite: >= 1 valid key per tile
-    const float a0 = ex2(m0 - mn0), a1 = ex2(m1 - mn1);
-    m0 = mn0;
-    m1 = mn1;
-    const float p0 = ex2(s0 - mn0), p1 = ex2(s1 - mn1), p2 = ex2(s2 - mn0), p3 = ex2(s3 - mn1);
+    // Lazy rescaling (as in the prefill tile): a head's reference max moves
+    // only when the stage max exceeds it by more than 8 (log2 units), so every
+    // weight is <= 2^8 and O and l are rescaled only then. Every stage has a
+    // valid key, so the first stage always sets the reference (alpha = 0).
+    const bool up0 = mx0 > m0 + 8.f, up1 = mx1 > m1 + 8.f;
+    if (__any_sync(0xffffffffu, up0 || up1)) {
+      float a0 = 1.f, a1 = 1.f;
+      if (up0) {
+        a0 = ex2(m0 - mx0);
+        m0 = mx0;
+      }
+      if (up1) {
+        a1 = ex2(m1 - mx1);
+        m1 = mx1;
+      }
+      l0 *= a0;
+      l1 *= a1;
+#pragma unroll
+      for (int mt = 0; mt < KS; ++mt) {
+        o[mt][0] *= a0;
+        o[mt][1] *= a1;
+        o[mt][2] *= a0;
+        o[mt][3] *= a1;
+      }
+    }
+    const float p0 = ex2(s0 - m0), p1 = ex2(s1 - m1), p2 = ex2(s2 - m0), p3 = ex2(s3 - m1);
     const uint32_t x01 = pack_bf16(p0, p1);  // key hrow
     const uint32_t x23 = pack_bf16(p2, p3);  // key hrow + 8
     // The normaliser sums the unrounded fp32 weights: summing the bf16-rounded
     // ones would put their rounding (2^-9 relative) straight into the LSE.
-    l0 = l0 * a0 + (p0 + p2);
-    l1 = l1 * a1 + (p1 + p3);
-#pragma unroll
-    for (int mt = 0; mt < KS; ++mt) {
-      o[mt][0] *= a0;
-      o[mt][1] *= a1;
-      o[mt][2] *= a0;
-      o[mt][3] *= a1;
-    }
+    l0 += p0 + p2;
+    l1 += p1 + p3;
     // P^T as the B operand: transpose each 8x8 (key x head) block.
     const uint32_t b0 = movmatrix_t(x01);
     const uint32_t b1 = movmatrix_t(x23);
