@@ -172,11 +172,10 @@ def test_pair_kernel_splits_the_tail_wave(harness):
     """Long-context prefill (64/8 heads, 1024 rows after 16384) on 74 CTA
     pairs: 256 pair units are 3.46 waves; splitting the units of the partial
     last wave in two shortens the finish time below that of no split and of
-    any uniform split, and the fused call (prefill the longer phase) does the
-    same."""
+    any uniform split."""
     pre, dec = [(16384, 1024)], [20000 + 900 * i for i in range(16)]
     for fused in (False, True):
-        p = plan(harness, 64, 8, pre, dec if fused else [], fused=fused, clusters=74)
+        p = plan(harness, 64, 8, pre, [], fused=fused, clusters=74)
         check_units(p, 64, 8, pre)
         splits = [u[4] for u in p["punits"]]
         n_split_units = len({(u[0], u[1], u[2]) for u in p["punits"] if u[4] > 1})
@@ -188,6 +187,25 @@ def test_pair_kernel_splits_the_tail_wave(harness):
         for s in (2, 3, 4):
             uniform = [(w * (k + 1)) // s - (w * k) // s for w in unsplit for k in range(s)]
             assert lpt_makespan(works, 74) <= lpt_makespan(uniform, 74)
+
+
+def test_fused_call_with_decodes_keeps_the_last_wave_whole(harness):
+    """One-SM tile, long-context batch: 256 units are 1.73 waves of 148 SMs.
+    A launch of the prefill alone splits the last wave's 108 units in four
+    (each SM then ends after 1.75 units of work, not 2); a fused launch that
+    carries the decodes keeps them whole, so the SMs the last wave leaves
+    free stream decode."""
+    pre, dec = [(16384, 1024)], [20000 + 900 * i for i in range(16)]
+    alone = plan(harness, 64, 8, pre, [], fused=False, clusters=0)
+    check_units(alone, 64, 8, pre)
+    parts = {}
+    for u in alone["punits"]:
+        parts.setdefault((u[0], u[1], u[2]), u[4])
+    assert sorted(parts.values()).count(4) == 256 - 148
+    assert sorted(parts.values()).count(1) == 148
+    fused = plan(harness, 64, 8, pre, dec, fused=True, clusters=0)
+    check_units(fused, 64, 8, pre)
+    assert {u[4] for u in fused["punits"]} == {1} and len(fused["punits"]) == 256
 
 
 def test_pair_kernel_maps_k_in_halves(harness):
