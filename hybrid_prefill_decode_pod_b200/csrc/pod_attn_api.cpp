@@ -70,7 +70,7 @@ struct DeviceGuard {
 // tables) start at zero.
 struct PlanLayout {
   size_t ctl, ticket, stats, tables0;                        // fixed part
-  size_t pgroup, dgroup, tables, preq, punits, dreq, dunit;  // capacities
+  size_t pgroup, dgroup, tables, preq, punits, dreq;  // capacities
   size_t end;
 };
 
@@ -88,6 +88,7 @@ struct pod_attn_ctx {
   int dec_turn = 1;      // decode units each warp claims per decode turn of a fused CTA
   int dec_split = 0;     // 0: cost model; else keys per decode split (multiple of 16)
   int pre_split = 0;     // 0: makespan model; else KV splits per prefill tile
+  bool tail_split_fused = false;  // ablation: also split the last wave in fused calls with decodes
   bool split_uncapped = false;  // forced splits ignore the two-wave cap (ablation)
   // prefill tile: a CTA pair on two SMs (M = 256, head_dim 128) or one SM
   bool use_pair = false;
@@ -119,7 +120,6 @@ struct pod_attn_ctx {
   std::vector<PrefillUnit> parts_tmp;
   std::vector<PrefillReq> preq_tmp;
   std::vector<DecodeReq> dreq_tmp;
-  std::vector<int> dunit_tmp;
 };
 
 namespace {
@@ -137,7 +137,6 @@ PlanLayout plan_layout(const pod_attn_ctx* c) {
   L.preq = o; o = align_up(o + sizeof(PrefillReq) * kMaxPrefillReqs, 64);
   L.punits = o; o = align_up(o + sizeof(PrefillUnit) * (size_t)c->cap_punits, 64);
   L.dreq = o; o = align_up(o + sizeof(DecodeReq) * (size_t)c->cap_dreqs, 64);
-  L.dunit = o; o = align_up(o + sizeof(int) * (size_t)c->cap_dunits, 64);
   L.end = o;
   return L;
 }
@@ -365,7 +364,8 @@ int build_plan(pod_attn_ctx* c, const pod_prefill_args* pa, const pod_decode_arg
       // unsplit last wave leaves free run decode turns instead, and the split
       // measured slower (B200, long-context batch: 725 us against 670 us
       // unsplit; prefill alone 587 us against 602 us).
-      const int tail = (n_draft > slots && !(fused_call && nd > 0)) ? n_draft % slots : 0;
+      const int tail =
+          (n_draft > slots && (c->tail_split_fused || !(fused_call && nd > 0))) ? n_draft % slots : 0;
       if (tail > 0) {
         // The tail units are the shortest, so their parts queue after every
         // unsplit unit: run the unsplit prefix once, then each tail split.
@@ -448,7 +448,6 @@ int build_plan(pod_attn_ctx* c, const pod_prefill_args* pa, const pod_decode_arg
   // ---- decode
   c->dreq_tmp.assign(nd, DecodeReq{});
   DecodeReq* dreq = c->dreq_tmp.data();
-  std::vector<int>& dunit = c->dunit_tmp;
   // Keys per decode split (a multiple of the 16-key decode tile): the
   // candidate minimising an estimate of the decode makespan on the persistent
   // decode warps. Units are claimed dynamically, so with U units of at most
@@ -490,7 +489,6 @@ int build_plan(pod_attn_ctx* c, const pod_prefill_args* pa, const pod_decode_arg
     }
   }
   int n_du = 0, n_dg = 0, n_ds = 0;
-  dunit.clear();
   for (int r = 0; r < nd; ++r) {
     DecodeReq& R = dreq[r];
     const int len = da->ctx_lens[r];
@@ -508,7 +506,6 @@ int build_plan(pod_attn_ctx* c, const pod_prefill_args* pa, const pod_decode_arg
     }
     const int nu = R.n_split * Hk;
     if (n_du + nu > c->cap_dunits) return POD_ECAPACITY;
-    dunit.insert(dunit.end(), nu, r);
     n_du += nu;
   }
   if (n_dg > c->cap_dgroups || n_ds > c->cap_dslots) return POD_ECAPACITY;
@@ -571,19 +568,18 @@ int build_plan(pod_attn_ctx* c, const pod_prefill_args* pa, const pod_decode_arg
   const size_t o_preq = align_up(o_dg + sizeof(int) * (size_t)n_dg, 64);
   const size_t o_pu = align_up(o_preq + sizeof(PrefillReq) * (size_t)np, 64);
   const size_t o_dreq = align_up(o_pu + sizeof(PrefillUnit) * (size_t)n_pu, 64);
-  const size_t o_du = align_up(o_dreq + sizeof(DecodeReq) * (size_t)nd, 64);
-  const size_t o_end = o_du + sizeof(int) * (size_t)n_du;
+  // (decode units are not listed: a unit finds its request by a search of
+  // the requests' first-unit indices, which ascend)
+  const size_t o_end = o_dreq + sizeof(DecodeReq) * (size_t)nd;
   if (o_end > c->plan_cap) return POD_ECAPACITY;
   std::memset(h, 0, o_preq);
   if (np) std::memcpy(h + o_preq, preq, sizeof(PrefillReq) * (size_t)np);
   if (n_pu) std::memcpy(h + o_pu, punits, sizeof(PrefillUnit) * (size_t)n_pu);
   if (nd) std::memcpy(h + o_dreq, dreq, sizeof(DecodeReq) * (size_t)nd);
-  if (n_du) std::memcpy(h + o_du, dunit.data(), sizeof(int) * (size_t)n_du);
   char* dp = c->d_plan;
   Q.preq = reinterpret_cast<const PrefillReq*>(dp + o_preq);
   Q.punits = reinterpret_cast<const PrefillUnit*>(dp + o_pu);
   Q.dreq = reinterpret_cast<const DecodeReq*>(dp + o_dreq);
-  Q.dunit_req = reinterpret_cast<const int*>(dp + o_du);
   if (np) {
     Q.q_p = static_cast<const uint16_t*>(pa->q);
     Q.o_p = static_cast<uint16_t*>(pa->o);
@@ -791,6 +787,8 @@ int pod_attn_create(pod_attn_ctx** out, const pod_attn_config* cfg) {
     c->split_uncapped = v < 0;
     c->pre_split = std::max(0, std::min(kMaxPrefillSplit, v < 0 ? -v : v));
   }
+  if (const char* e = std::getenv("POD_ATTN_TAIL_SPLIT_FUSED"))
+    c->tail_split_fused = std::atoi(e) != 0;
   if (const char* e = std::getenv("POD_ATTN_DEC_SPLIT"))
     c->dec_split = std::max(0, std::atoi(e)) / kDecTile * kDecTile;
   // The one-SM prefill tile serves every head_dim by default: it measured

@@ -256,6 +256,22 @@ POD_DEV void merge_decode_group(const Plan& P, const DecodeReq& R, int r, int g,
                           P.lse_d + (size_t)r * P.H + (size_t)g * P.G, 1, lane);
 }
 
+// The request of decode unit u: the last request whose first unit is <= u.
+// Requests own consecutive unit ranges (n_split x Hk units each, never empty)
+// in request order, so the per-request table replaces a per-unit one and the
+// plan a call copies grows with its requests, not with its units.
+POD_DEV int decode_unit_request(const Plan& P, int u) {
+  int lo = 0, hi = P.n_decode_reqs - 1;  // dreq[lo].unit0 <= u throughout
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(&P.dreq[mid].unit0) <= u)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  return lo;
+}
+
 // ============================================================= decode unit
 // One warp, one unit (request r, KV head g, keys [kbeg, kend)). The ring of
 // `NST` stages lives at `wsm` (each stage: 16 K rows then 16 V rows, padded).
@@ -279,7 +295,7 @@ POD_DEV bool decode_unit_warp(const Plan& P, int u, uint8_t* wsm, uint32_t& ring
   constexpr int CH = D * 2 / 16;  // 16-byte pieces per row
   constexpr int RPI = 32 / CH;    // rows per warp instruction
   static_assert(2 * kDecTile % RPI == 0, "a stage is a whole number of warp instructions");
-  const int r = P.dunit_req[u];
+  const int r = decode_unit_request(P, u);
   const DecodeReq R = P.dreq[r];
   const int Hk = P.Hk, G = P.G;
   const int local = u - R.unit0;

@@ -83,8 +83,7 @@ struct Plan {
   long long wait_budget;         // cycles a bounded wait may spin
   const PrefillReq* preq;
   const PrefillUnit* punits;
-  const DecodeReq* dreq;
-  const int* dunit_req;          // request of each decode unit
+  const DecodeReq* dreq;         // unit0 ascending: a unit's request is found by search
   const uint16_t* q_p; uint16_t* o_p; float* lse_p;
   const uint16_t* q_d; uint16_t* o_d; float* lse_d;
   const int* bt_p; const int* bt_d;

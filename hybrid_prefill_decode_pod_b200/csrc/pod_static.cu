@@ -41,13 +41,13 @@ constexpr int kMaxKvHeads = POD_STATIC_MAX_KV_HEADS;
 constexpr int kMaxDim = 128;
 
 // Byte layout of the scratch array. The head part (control words, merge
-// counters, request table, unit table) is rewritten by every call; the
-// partial results are written before they are read.
+// counters, request table) is rewritten by every call; the partial results
+// are written before they are read. (A decode unit finds its request by a
+// search of the requests' first-unit indices: there is no unit table.)
 constexpr size_t kCtlOff = 0;                                        // 16 ints
 constexpr size_t kGroupOff = 256;                                    // merge counters
 constexpr size_t kReqOff = kGroupOff + sizeof(int) * kMaxReqs * kMaxKvHeads;
-constexpr size_t kUnitOff = kReqOff + sizeof(DecodeReq) * kMaxReqs;
-constexpr size_t kHeadBytes = kUnitOff + sizeof(int) * kMaxUnits;
+constexpr size_t kHeadBytes = kReqOff + sizeof(DecodeReq) * kMaxReqs;
 constexpr size_t kLseOff = (kHeadBytes + 255) / 256 * 256;
 constexpr size_t kPartOff = kLseOff + sizeof(float) * kMaxUnits * kMaxGroup;
 constexpr size_t kScratchBytes = kPartOff + sizeof(float) * kMaxUnits * kMaxGroup * kMaxDim;
@@ -157,11 +157,10 @@ extern "C" POD_API int pod_attn_decode_static(int num_qo_heads, int num_kv_heads
   if (rc) return rc;
 
   // head part of the scratch: zeroed control words and merge counters, then
-  // the request table and the unit -> request table
+  // the request table
   std::lock_guard<std::mutex> lk(g_mu);
   std::memset(g_host_head, 0, kReqOff);
   DecodeReq* req = reinterpret_cast<DecodeReq*>(g_host_head + kReqOff);
-  int* unit_req = reinterpret_cast<int*>(g_host_head + kUnitOff);
   int n_units = 0, n_groups = 0, n_slots = 0;
   for (int r = 0; r < a->num_reqs; ++r) {
     DecodeReq& R = req[r];
@@ -178,10 +177,9 @@ extern "C" POD_API int pod_attn_decode_static(int num_qo_heads, int num_kv_heads
       n_groups += Hk;
       n_slots += R.n_split * Hk;
     }
-    for (int i = 0; i < R.n_split * Hk; ++i) unit_req[n_units + i] = r;
     n_units += R.n_split * Hk;
   }
-  const size_t head_bytes = kUnitOff + sizeof(int) * (size_t)n_units;
+  const size_t head_bytes = kReqOff + sizeof(DecodeReq) * (size_t)a->num_reqs;
   if (cudaMemcpyAsync(st->scratch, g_host_head, head_bytes, cudaMemcpyHostToDevice, s) !=
       cudaSuccess)
     return POD_ECUDA;
@@ -206,7 +204,6 @@ extern "C" POD_API int pod_attn_decode_static(int num_qo_heads, int num_kv_heads
   // over from an earlier call.
   P.flags = kFlagPoisonOnStatus;
   P.dreq = reinterpret_cast<const DecodeReq*>(st->scratch + kReqOff);
-  P.dunit_req = reinterpret_cast<const int*>(st->scratch + kUnitOff);
   P.q_d = static_cast<const uint16_t*>(a->q);
   P.o_d = static_cast<uint16_t*>(a->o);
   P.lse_d = a->lse;

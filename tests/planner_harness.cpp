@@ -159,13 +159,11 @@ int main(int argc, char** argv) {
     const PrefillReq* preq = reinterpret_cast<const PrefillReq*>(at(P.preq));
     const PrefillUnit* pu = reinterpret_cast<const PrefillUnit*>(at(P.punits));
     const DecodeReq* dreq = reinterpret_cast<const DecodeReq*>(at(P.dreq));
-    const int* du = reinterpret_cast<const int*>(at(P.dunit_req));
     // every table lies inside the bytes the call copies, and the zeroed words
     // (queue heads, tickets, merge counters) are zero
-    const size_t ends[4] = {(size_t)((const char*)(P.preq + np) - c.d_plan),
+    const size_t ends[3] = {(size_t)((const char*)(P.preq + np) - c.d_plan),
                             (size_t)((const char*)(P.punits + P.n_prefill_units) - c.d_plan),
-                            (size_t)((const char*)(P.dreq + nd) - c.d_plan),
-                            (size_t)((const char*)(P.dunit_req + P.n_decode_units) - c.d_plan)};
+                            (size_t)((const char*)(P.dreq + nd) - c.d_plan)};
     bool inside = true;
     for (size_t e : ends) inside = inside && e <= bytes && e <= c.plan_cap;
     bool zeroed = true;
@@ -198,8 +196,13 @@ int main(int argc, char** argv) {
       std::printf("%s{\"len\": %d, \"n_split\": %d, \"unit0\": %d, \"group0\": %d, \"slot0\": %d}",
                   i ? ", " : "", dreq[i].len, dreq[i].n_split, dreq[i].unit0, dreq[i].group0,
                   dreq[i].slot0);
+    // the request of each decode unit, by the rule the kernel applies (the
+    // last request whose first unit is <= u)
     std::printf("], \"dunit\": [");
-    for (int u = 0; u < P.n_decode_units; ++u) std::printf("%s%d", u ? ", " : "", du[u]);
+    for (int u = 0, r = 0; u < P.n_decode_units; ++u) {
+      while (r + 1 < nd && dreq[r + 1].unit0 <= u) ++r;
+      std::printf("%s%d", u ? ", " : "", r);
+    }
     std::printf("]");
   }
   std::printf("}\n");
