@@ -790,7 +790,7 @@ int pod_attn_create(pod_attn_ctx** out, const pod_attn_config* cfg) {
   if (const char* e = std::getenv("POD_ATTN_TAIL_SPLIT_FUSED"))
     c->tail_split_fused = std::atoi(e) != 0;
   if (const char* e = std::getenv("POD_ATTN_DEC_SPLIT"))
-    c->dec_split = std::max(0, std::atoi(e)) / kDecTile * kDecTile;
+    c->dec_split = std::max(0, std::atoi(e)) / dec_stage_keys(D) * dec_stage_keys(D);
   // The one-SM prefill tile serves every head_dim by default: it measured
   // faster than the CTA-pair tile on every hybrid workload of the benchmark
   // (the pair's single MMA-issuing thread sets its pace). The pair tile

@@ -107,7 +107,7 @@ struct FusedLayout {
   static constexpr int V_OFF = K_OFF + kPrefillStages * KT;     // V ring
   static constexpr int PREFILL_END = V_OFF + kPrefillStages * KT;
   static constexpr int DEC_ROW = D * 2 + 16;  // padded row: conflict-free ldmatrix
-  static constexpr int DEC_STAGE = 2 * kDecTile * DEC_ROW;
+  static constexpr int DEC_STAGE = 2 * dec_stage_keys(D) * DEC_ROW;
   static constexpr int DEC_WARP = kFusedDecStages * DEC_STAGE;
   static constexpr int DEC_END = kFusedDecWarps * DEC_WARP;  // decode turns overlay prefill
   static constexpr int SIDE_OFF = PREFILL_END > DEC_END ? PREFILL_END : DEC_END;
@@ -137,7 +137,7 @@ struct FusedLayout {
 template <int D>
 struct DecodeLayout {
   static constexpr int ROW = D * 2 + 16;
-  static constexpr int STAGE = 2 * kDecTile * ROW;
+  static constexpr int STAGE = 2 * dec_stage_keys(D) * ROW;
   static constexpr int WARP = kDecodeStages * STAGE;
   static constexpr int FLAG_OFF = kDecodeWarps * WARP;  // one abort flag per warp
   static constexpr int SMEM_BYTES = FLAG_OFF + kDecodeWarps * 4;
@@ -290,11 +290,13 @@ POD_DEV bool decode_unit_warp(const Plan& P, int u, uint8_t* wsm, uint32_t& ring
                               bool inline_merge, volatile int* abort_flag) {
   static_assert(NST >= 1 && NST <= 8, "cp.async.wait_group counts at most 7 pending groups");
   constexpr int ROW = D * 2 + 16;
-  constexpr int STAGE = 2 * kDecTile * ROW;
+  constexpr int NB = dec_stage_blocks(D);  // 16-key mma blocks per stage
+  constexpr int KPS = kDecTile * NB;       // keys per stage
+  constexpr int STAGE = 2 * KPS * ROW;     // K rows 0..KPS-1, then V rows
   constexpr int KS = D / 16;
   constexpr int CH = D * 2 / 16;  // 16-byte pieces per row
   constexpr int RPI = 32 / CH;    // rows per warp instruction
-  static_assert(2 * kDecTile % RPI == 0, "a stage is a whole number of warp instructions");
+  static_assert(kDecTile % RPI == 0, "a block is a whole number of warp instructions");
   const int r = decode_unit_request(P, u);
   const DecodeReq R = P.dreq[r];
   const int Hk = P.Hk, G = P.G;
@@ -303,7 +305,7 @@ POD_DEV bool decode_unit_warp(const Plan& P, int u, uint8_t* wsm, uint32_t& ring
   const int g = local - s * Hk;
   const int kbeg = s * P.dec_split_len;
   const int kend = min(R.len, kbeg + P.dec_split_len);
-  const int n_tiles = (kend - kbeg + kDecTile - 1) / kDecTile;
+  const int n_tiles = (kend - kbeg + KPS - 1) / KPS;  // stages
   const int q4 = lane & 3;
   const int hrow = lane >> 2;  // query head within the group (B column / C row of S^T)
 
@@ -331,45 +333,50 @@ POD_DEV bool decode_unit_warp(const Plan& P, int u, uint8_t* wsm, uint32_t& ring
 #endif
   const int col = lane % CH, rsub = lane / CH;  // this lane's piece and row phase
 
-  // Stage t: keys kbeg + 16 t .. +15 (a ragged tail re-reads the last valid
-  // row; those keys are masked below). Split lengths are multiples of 16, so
-  // a stage never crosses a 16-token page: one block-table entry per stage.
+  // Stage t: keys kbeg + KPS t .. +KPS-1, in 16-key blocks (a ragged tail
+  // re-reads the last valid row; those keys are masked below). Split lengths
+  // are multiples of KPS, so a block never crosses a 16-token page: one
+  // block-table entry per block.
   auto issue = [&](int t) {
     const uint32_t st = (ring + t) % NST;
-    const int key0 = kbeg + t * kDecTile;
-    size_t base_off;
-    if (P.paged) {
-      int phys = __ldg(P.bt_d + (size_t)R.bt_row * P.bt_stride_d + (key0 >> 4));
-      phys = min(max(phys, 0), P.pool_blocks - 1);  // never read outside the pool
-      base_off = (size_t)phys * kDecTile * row_elems + (size_t)g * D;
-    } else {
-      base_off = (size_t)key0 * row_elems + (size_t)g * D;
-    }
-    const int last = kend - 1 - key0;  // last valid key of the stage, 0..15
-    // this lane's piece of key rows rsub, rsub + RPI, ... of K (then V)
-    const uint32_t dk = wsm_a + st * STAGE + rsub * ROW + col * 16;
-    const uint16_t* sk = kbase + base_off + col * 8;
-    const uint16_t* sv = vbase + base_off + col * 8;
 #if POD_L2_HINTS
 #define POD_DEC_COPY(d, s) cp_async16_hint(d, s, once)
 #else
 #define POD_DEC_COPY(d, s) cp_async16(d, s)
 #endif
-    if (last >= kDecTile - 1) {  // a full stage: rows advance by RPI rows of the cache
-      const size_t step = (size_t)RPI * row_elems;
-      sk += (size_t)rsub * row_elems;
-      sv += (size_t)rsub * row_elems;
 #pragma unroll
-      for (int i = 0; i < kDecTile / RPI; ++i, sk += step, sv += step) {
-        POD_DEC_COPY(dk + i * RPI * ROW, sk);
-        POD_DEC_COPY(dk + (kDecTile + i * RPI) * ROW, sv);
+    for (int bk = 0; bk < NB; ++bk) {
+      // a block wholly past the end re-reads the last valid row as well
+      const int key0 = min(kbeg + t * KPS + bk * kDecTile, kend - 1) & ~(kDecTile - 1);
+      size_t base_off;
+      if (P.paged) {
+        int phys = __ldg(P.bt_d + (size_t)R.bt_row * P.bt_stride_d + (key0 >> 4));
+        phys = min(max(phys, 0), P.pool_blocks - 1);  // never read outside the pool
+        base_off = (size_t)phys * kDecTile * row_elems + (size_t)g * D;
+      } else {
+        base_off = (size_t)key0 * row_elems + (size_t)g * D;
       }
-    } else {  // the ragged tail re-reads the last valid row (masked in the softmax)
+      const int last = kend - 1 - key0;  // last valid key of the block (>= 0)
+      // this lane's piece of key rows rsub, rsub + RPI, ... of K (then V)
+      const uint32_t dk = wsm_a + st * STAGE + (bk * kDecTile + rsub) * ROW + col * 16;
+      const uint16_t* sk = kbase + base_off + col * 8;
+      const uint16_t* sv = vbase + base_off + col * 8;
+      if (last >= kDecTile - 1) {  // a full block: rows advance by RPI rows of the cache
+        const size_t step = (size_t)RPI * row_elems;
+        sk += (size_t)rsub * row_elems;
+        sv += (size_t)rsub * row_elems;
 #pragma unroll
-      for (int i = 0; i < kDecTile / RPI; ++i) {
-        const size_t k = (size_t)min(i * RPI + rsub, last) * row_elems;
-        POD_DEC_COPY(dk + i * RPI * ROW, sk + k);
-        POD_DEC_COPY(dk + (kDecTile + i * RPI) * ROW, sv + k);
+        for (int i = 0; i < kDecTile / RPI; ++i, sk += step, sv += step) {
+          POD_DEC_COPY(dk + i * RPI * ROW, sk);
+          POD_DEC_COPY(dk + (KPS + i * RPI) * ROW, sv);
+        }
+      } else {  // the ragged tail re-reads the last valid row (masked in the softmax)
+#pragma unroll
+        for (int i = 0; i < kDecTile / RPI; ++i) {
+          const size_t k = (size_t)min(i * RPI + rsub, last) * row_elems;
+          POD_DEC_COPY(dk + i * RPI * ROW, sk + k);
+          POD_DEC_COPY(dk + (KPS + i * RPI) * ROW, sv + k);
+        }
       }
     }
 #undef POD_DEC_COPY
@@ -395,27 +402,37 @@ POD_DEV bool decode_unit_warp(const Plan& P, int u, uint8_t* wsm, uint32_t& ring
       ok = false;
       break;
     }
-    const uint32_t kb = wsm_a + st * STAGE;
-    const uint32_t vb = kb + kDecTile * ROW;
-    // S^T[16 keys x 8 heads]
-    // two independent accumulator chains halve the dependent mma latency
-    float c[4] = {0.f, 0.f, 0.f, 0.f}, c2[4] = {0.f, 0.f, 0.f, 0.f};
+    const uint32_t kb0 = wsm_a + st * STAGE;
+    const uint32_t vb0 = kb0 + KPS * ROW;
+    // S^T[16 keys x 8 heads] per block; the G query heads of the KV group
+    // are the mma N dimension. Lane: keys hrow and hrow + 8 of each block,
+    // heads 2 q4 and 2 q4 + 1.
+    float sv[NB][4];
 #pragma unroll
-    for (int kk = 0; kk < KS; kk += 2) {
-      uint32_t a[4], a2[4];
-      ldsm_x4(kb + (lane & 15) * ROW + (kk * 16 + 8 * (lane >> 4)) * 2, a);
-      ldsm_x4(kb + (lane & 15) * ROW + ((kk + 1) * 16 + 8 * (lane >> 4)) * 2, a2);
-      mma_16816(c, a, qb[kk][0], qb[kk][1]);
-      mma_16816(c2, a2, qb[kk + 1][0], qb[kk + 1][1]);
+    for (int bk = 0; bk < NB; ++bk) {
+      const uint32_t kb = kb0 + bk * kDecTile * ROW;
+      // two independent accumulator chains halve the dependent mma latency
+      float c[4] = {0.f, 0.f, 0.f, 0.f}, c2[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int kk = 0; kk < KS; kk += 2) {
+        uint32_t a[4], a2[4];
+        ldsm_x4(kb + (lane & 15) * ROW + (kk * 16 + 8 * (lane >> 4)) * 2, a);
+        ldsm_x4(kb + (lane & 15) * ROW + ((kk + 1) * 16 + 8 * (lane >> 4)) * 2, a2);
+        mma_16816(c, a, qb[kk][0], qb[kk][1]);
+        mma_16816(c2, a2, qb[kk + 1][0], qb[kk + 1][1]);
+      }
+      const int key_a = kbeg + t * KPS + bk * kDecTile + hrow;
+      sv[bk][0] = (key_a < kend) ? (c[0] + c2[0]) * sc : -INFINITY;
+      sv[bk][1] = (key_a < kend) ? (c[1] + c2[1]) * sc : -INFINITY;
+      sv[bk][2] = (key_a + 8 < kend) ? (c[2] + c2[2]) * sc : -INFINITY;
+      sv[bk][3] = (key_a + 8 < kend) ? (c[3] + c2[3]) * sc : -INFINITY;
     }
+    float mx0 = fmaxf(sv[0][0], sv[0][2]), mx1 = fmaxf(sv[0][1], sv[0][3]);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) c[i] += c2[i];
-    const int key_a = kbeg + t * kDecTile + hrow;
-    float s0 = (key_a < kend) ? c[0] * sc : -INFINITY;
-    float s1 = (key_a < kend) ? c[1] * sc : -INFINITY;
-    float s2 = (key_a + 8 < kend) ? c[2] * sc : -INFINITY;
-    float s3 = (key_a + 8 < kend) ? c[3] * sc : -INFINITY;
-    float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
+    for (int bk = 1; bk < NB; ++bk) {
+      mx0 = max3(mx0, sv[bk][0], sv[bk][2]);
+      mx1 = max3(mx1, sv[bk][1], sv[bk][3]);
+    }
 #pragma unroll
     for (int off = 4; off < 32; off <<= 1) {
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
@@ -446,22 +463,26 @@ POD_DEV bool decode_unit_warp(const Plan& P, int u, uint8_t* wsm, uint32_t& ring
         o[mt][3] *= a1;
       }
     }
-    const float p0 = ex2(s0 - m0), p1 = ex2(s1 - m1), p2 = ex2(s2 - m0), p3 = ex2(s3 - m1);
-    const uint32_t x01 = pack_bf16(p0, p1);  // key hrow
-    const uint32_t x23 = pack_bf16(p2, p3);  // key hrow + 8
-    // The normaliser sums the unrounded fp32 weights: summing the bf16-rounded
-    // ones would put their rounding (2^-9 relative) straight into the LSE.
-    l0 += p0 + p2;
-    l1 += p1 + p3;
-    // P^T as the B operand: transpose each 8x8 (key x head) block.
-    const uint32_t b0 = movmatrix_t(x01);
-    const uint32_t b1 = movmatrix_t(x23);
 #pragma unroll
-    for (int mt = 0; mt < KS; ++mt) {
-      uint32_t a[4];
-      ldsm_x4_t(vb + ((lane & 7) + 8 * (lane >> 4)) * ROW + (mt * 16 + 8 * ((lane >> 3) & 1)) * 2,
-                a);
-      mma_16816(o[mt], a, b0, b1);
+    for (int bk = 0; bk < NB; ++bk) {
+      const float p0 = ex2(sv[bk][0] - m0), p1 = ex2(sv[bk][1] - m1);
+      const float p2 = ex2(sv[bk][2] - m0), p3 = ex2(sv[bk][3] - m1);
+      // The normaliser sums the unrounded fp32 weights: summing the
+      // bf16-rounded ones would put their rounding (2^-9 relative) straight
+      // into the LSE.
+      l0 += p0 + p2;
+      l1 += p1 + p3;
+      // P^T as the B operand: transpose each 8x8 (key x head) block.
+      const uint32_t b0 = movmatrix_t(pack_bf16(p0, p1));  // key hrow
+      const uint32_t b1 = movmatrix_t(pack_bf16(p2, p3));  // key hrow + 8
+      const uint32_t vb = vb0 + bk * kDecTile * ROW;
+#pragma unroll
+      for (int mt = 0; mt < KS; ++mt) {
+        uint32_t a[4];
+        ldsm_x4_t(vb + ((lane & 7) + 8 * (lane >> 4)) * ROW + (mt * 16 + 8 * ((lane >> 3) & 1)) * 2,
+                  a);
+        mma_16816(o[mt], a, b0, b1);
+      }
     }
     __syncwarp();  // every lane's reads of this stage are done before its refill
     if (t + NST < n_tiles) {

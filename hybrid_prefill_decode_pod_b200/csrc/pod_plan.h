@@ -18,7 +18,12 @@ constexpr int kMaxPrefillReqs = 16;
 constexpr int kQTile = 128;           // prefill query rows per unit (= UMMA M)
 constexpr int kKVTile = 128;          // prefill keys per KV tile (= UMMA N of S)
 constexpr int kPrefillStages = 2;     // K/V smem ring depth in the prefill role
-constexpr int kDecTile = 16;          // decode keys per staged tile (= mma M)
+constexpr int kDecTile = 16;          // decode keys per mma block (= mma M)
+// Keys per decode stage: one 16-key block at d = 128, two at d = 64, so a
+// stage moves the same bytes (8 KB) and its fixed per-stage work (waits, row
+// maxima, exponentials, transposes) is spread over as many bytes.
+constexpr int dec_stage_blocks(int D) { return D == 64 ? 2 : 1; }
+constexpr int dec_stage_keys(int D) { return kDecTile * dec_stage_blocks(D); }
 constexpr int kRoleWarps = 10;        // 8 softmax (2 query tiles) + MMA issuer + TMA producer;
                                       // all of them run decode units in a decode turn
 constexpr int kSideDecWarps = 2;      // warps that stream decode units for the CTA's whole life,
