@@ -9,13 +9,15 @@
 //    softmax warps (one thread per query row = TMEM lane) run the online
 //    softmax of the two tiles in ping-pong with the tensor pipe.
 //  * decode unit: one warp (a "virtual decode CTA", paper §4.2.3) streams the
-//    K/V rows of (request, KV head, key split) with TMA bulk copies into a
-//    padded smem ring and runs S^T = K Q^T and O^T += V^T P^T on the legacy
-//    m16n8k16 tensor-core path with the G query heads of the group as N = 8
-//    (the paper's small decode tile, §4.2.1).
+//    K/V rows of (request, KV head, key split) with 16-byte cp.async copies
+//    into a padded smem ring and runs S^T = K Q^T and O^T += V^T P^T on the
+//    legacy m16n8k16 tensor-core path with the G query heads of the group as
+//    N = 8 (the paper's small decode tile, §4.2.1). A claimed unit finds its
+//    request by a search of the requests' first-unit indices.
 //  * merge: log-sum-exp combination of split partials, in split order.
-//  * fused kernel: one persistent 12-warp CTA per SM. Its ten role warps read
-//    %smid, take a ticket from that SM's counter and pick prefill or decode
+//  * fused kernel: one persistent 12-warp CTA per SM (the CTA-pair kernel
+//    further down runs the same roles on clusters of two). Its ten role warps
+//    read %smid, take a ticket from that SM's counter and pick prefill or decode
 //    work (§4.1 SM-aware scheduling, §4.4 persistent threads, §5.4.2 role
 //    allocation); its two side warps stream decode units for the CTA's whole
 //    life, beside a prefill unit. The last CTA (or warp) to finish a split
@@ -35,10 +37,10 @@ namespace pod {
 // Share of the prefill softmax's exponentials evaluated by exp2_poly on the
 // FMA pipe instead of MUFU (pairs out of 8), and the bf16 packing used for P.
 // Measured on B200 (long-context prefill, 64/8 heads, d 128, two query tiles
-// per CTA): 0 pairs is fastest; 1/2/3/4 pairs cost 1.3x-1.6x, and replacing
-// every ex2 by a one-cycle stand-in changed nothing, so this softmax is bound
-// by issue and latency (and by the MMA hand-offs), not by MUFU. cvt packing
-// (round to nearest even) is 3 % faster than the integer round-half-away one.
+// per CTA): 0 pairs is fastest; 1 and 2 pairs cost 1.17x and 1.28x, since the
+// polynomial takes more FMA-pipe time per element than ex2 takes on MUFU.
+// cvt packing (round to nearest even) is 3 % faster than the integer
+// round-half-away one.
 #ifndef POD_SOFT_EXP2_PAIRS
 #define POD_SOFT_EXP2_PAIRS 0
 #endif
@@ -51,9 +53,10 @@ constexpr int kSoftPairs = POD_SOFT_EXP2_PAIRS;
 #define POD_PACK(a, b) pack_bf16(a, b)
 #endif
 
-// L2 cache-policy hints on the bulk loads: prefill K/V evict-last (several
-// query tiles re-read each tile), decode K/V evict-first (read once), so the
-// decode stream of a fused launch does not push the prefill's tiles out of L2.
+// L2 cache-policy hints: the decode K/V copies are evict-first (read once), so
+// the decode stream of a fused launch does not push the prefill's K/V tiles
+// (re-read by several query tiles) out of L2; the CTA-pair tile's K/V loads
+// are also marked evict-last (on the one-SM tile that measured no gain).
 #ifndef POD_L2_HINTS
 #define POD_L2_HINTS 1
 #endif

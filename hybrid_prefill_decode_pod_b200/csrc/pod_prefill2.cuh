@@ -22,10 +22,12 @@
 // its S is gone.
 //
 // Warps of each CTA (12):
-//   0-7   softmax: warp w serves TMEM lanes 32 (w % 4) .. +31 (its rows) and
-//         keys 64 (w / 4) .. +63 of every KV tile (the two warps of a row
-//         exchange the row max through shared memory), O columns 64 (w / 4)
-//         .. +63 in the rescale and the epilogue
+//   0-7   softmax: warp w serves TMEM lanes 32 (w % 4) .. +31 (its rows) on
+//         the KV tiles t with t % 2 == w / 4, all 128 keys of each; the lazily
+//         raised reference max passes from the owner of tile t to the owner of
+//         tile t + 1 through shared memory. Each warp rescales all of O when
+//         its rows' reference moves, and writes O columns 64 (w / 4) .. +63 in
+//         the epilogue
 //   8     leader CTA: one thread issues the pair MMAs; peer CTA: idle
 //   9     TMA producer: this CTA's query tile, K halves, V halves
 //   10-11 stream decode units for the CTA's whole life

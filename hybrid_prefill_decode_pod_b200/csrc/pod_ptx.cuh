@@ -1,5 +1,6 @@
-// pod_ptx.cuh -- thin inline-PTX wrappers for sm_100a (mbarrier, TMA, bulk
-// copies, tcgen05 MMA / TMEM, legacy warp MMA for the decode path).
+// pod_ptx.cuh -- thin inline-PTX wrappers for sm_100a (mbarrier, TMA tensor
+// copies, cp.async, tcgen05 MMA / TMEM, clusters, legacy warp MMA for the
+// decode path).
 #pragma once
 #include <cuda.h>
 #include <stdint.h>
