@@ -67,7 +67,7 @@ def test_reference_arm_under_torchrun_prints_one_line_from_rank0():
     cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
            "--master-addr", "127.0.0.1", "--master-port", str(_free_port()),
            os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
-           "--steps", "1", "--warmup", "3", "--workload", "tiny", "--ref-step-seconds", "0.2"]
+           "--steps", "2", "--warmup", "3", "--workload", "tiny", "--ref-budget-seconds", "30"]
     env = dict(os.environ, OMP_NUM_THREADS="2")
     p = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=540)
     assert p.returncode == 0, p.stderr[-2000:]
@@ -78,3 +78,5 @@ def test_reference_arm_under_torchrun_prints_one_line_from_rank0():
     assert d["value"] > 0 and d["unit"] == "us/call" and d["higher_is_better"] is False
     assert d["cpu_baseline"]["kind"] == "oracle"
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
+    # full oracle calls, the steps that ran reported as such
+    assert d["steps"] == 2 and d["warmup"] == 0 and "unsampled" in d["cpu_baseline"]["sample"]
