@@ -42,7 +42,7 @@ METRIC = "hybrid attention µs/call & % of max(FLOP,HBM) roofline vs serial P+D,
 UNIT = "us/call"
 DEFAULT_WORKLOAD = "long_context"
 # the other full-size configurations, timed in the same run as extra keys
-EXTRA_WORKLOADS = ("llama3_8b", "decode_heavy", "paged",
+EXTRA_WORKLOADS = ("tiny", "llama3_8b", "decode_heavy", "paged",
                    # shape variants: multi-head, group of 8, head_dim 64, many small chunks
                    "llama2_7b_mha", "yi6b_g8", "d64_mix", "many_chunks")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
