@@ -56,8 +56,10 @@ def test_scaled_shapes_match_oracle(shape, mode):
     compare(ref, out)
 
 
-def test_paged_matches_contiguous_bitwise_and_oracle():
-    b = W.make_custom(8, 2, 128, [(333, 190), (0, 40)], [1, 16, 17, 999, 2500], seed=9,
+@pytest.mark.parametrize("d", [128, 64])
+def test_paged_matches_contiguous_bitwise_and_oracle(d):
+    # d = 64 decode stages hold two 16-key blocks, so a stage spans two pages
+    b = W.make_custom(8, 2, d, [(333, 190), (0, 40)], [1, 16, 17, 33, 999, 2500], seed=9,
                       paged=True)
     ref = oracle.hybrid(b)
     paged, _ = run(b, "fused", paged=True)
