@@ -53,6 +53,13 @@ constexpr int kSoftPairs = POD_SOFT_EXP2_PAIRS;
 #define POD_PACK(a, b) pack_bf16(a, b)
 #endif
 
+// Softmax form of the one-SM prefill tile: 0 = one warp per query row and tile
+// (warps 0-3 tile 0, 4-7 tile 1); 1 = two warps per row splitting its keys,
+// all eight warps serving both tiles in turn.
+#ifndef POD_SOFTMAX_SPLIT
+#define POD_SOFTMAX_SPLIT 0
+#endif
+
 // L2 cache-policy hints: the decode K/V copies are evict-first (read once), so
 // the decode stream of a fused launch does not push the prefill's K/V tiles
 // (re-read by several query tiles) out of L2; the CTA-pair tile's K/V loads
@@ -115,6 +122,13 @@ struct FusedLayout {
   static constexpr int DEC_END = kFusedDecWarps * DEC_WARP;  // decode turns overlay prefill
   static constexpr int SIDE_OFF = PREFILL_END > DEC_END ? PREFILL_END : DEC_END;
   static constexpr int DATA_END = SIDE_OFF + kSideDecWarps * DEC_WARP;  // side decode rings
+  // The key-split softmax exchanges, per query row, four floats (two tiles x two
+  // key halves) through the 16-byte padding that ends every row of the side
+  // decode rings (the decode copies and ldmatrix reads stay in the row's first
+  // 2 D bytes); one row of padding per query row.
+  static constexpr int XCH_OFF = SIDE_OFF + D * 2;
+  static constexpr int XCH_STRIDE = DEC_ROW;
+  static_assert(kSideDecWarps * DEC_WARP / DEC_ROW >= kQTile, "one padded ring row per query row");
   static constexpr int BAR_OFF = (DATA_END + 127) & ~127;
   // barrier indices
   static constexpr int B_Q = 0;                         // Q0 and Q1 landed
@@ -593,7 +607,8 @@ __global__ void __launch_bounds__(kFusedThreads, kFusedSlotsPerSm)
   if (tid == 0) {
     for (int i = 0; i < L::N_BARS; ++i) {
       uint32_t cnt = 1;
-      if (i == L::B_PF || i == L::B_PF + 1) cnt = kSoftmaxWarps / 2;  // one per softmax warp
+      if (i == L::B_PF || i == L::B_PF + 1)  // one arrival per softmax warp of the tile
+        cnt = POD_SOFTMAX_SPLIT ? kSoftmaxWarps : kSoftmaxWarps / 2;
       mbar_init(bars + i * 8, cnt);
     }
     fence_mbar_init();
@@ -674,7 +689,11 @@ __global__ void __launch_bounds__(kFusedThreads, kFusedSlotsPerSm)
       if (role == 1) {
         const PrefillRange pr = prefill_range(P, unit);
         if (warp < kSoftmaxWarps) {
+#if POD_SOFTMAX_SPLIT
+          prefill_softmax_split<D>(P, pr, sm, tmem, ps, tid, abort_flag, misc + 7);
+#else
           prefill_softmax<D>(P, pr, sm, tmem, ps, tid, abort_flag, misc + 7);
+#endif
         } else if (warp == kSoftmaxWarps) {
           if (lane == 0) {
             issued_mma = true;

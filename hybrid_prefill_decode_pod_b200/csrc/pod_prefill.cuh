@@ -229,6 +229,284 @@ POD_DEV bool prefill_mma(const Plan& P, const PrefillRange& pr, uint8_t* sm, uin
   return true;
 }
 
+// ---- softmax + epilogue, key-split form (POD_SOFTMAX_SPLIT): warps w and
+// w + 4 share TMEM lane quarter w & 3 (query rows 32 (w & 3) .. +31) and split
+// every 128-key S row: warp w takes keys 0..63, warp w + 4 keys 64..127. All
+// eight warps serve tile 0 and then tile 1 of each KV step, so both warps of a
+// scheduler partition feed its MUFU with the same tile instead of two tiles
+// contending for it. The two halves of a row meet twice per tile:
+//   - the half-row maxima, through a 16-byte shared-memory slot per row and a
+//     named barrier of the 64 threads of the warp pair; both warps then hold
+//     the same row max, reference max and rescale decision;
+//   - at the end of the unit, the two partial row sums.
+// Each warp writes the P columns of its own keys (P of keys 64 h .. +63 goes to
+// S columns 32 h .. +31; the pair barrier orders that store after the other
+// warp's S load) and rescales and stores its half of O's columns.
+template <int D>
+POD_DEV bool prefill_softmax_split(const Plan& P, const PrefillRange& pr, uint8_t* sm,
+                                   uint32_t tmem, PipeState& ps, int tid,
+                                   volatile int* abort_flag, int* s_flag) {
+  using L = FusedLayout<D>;
+  constexpr int OB = D / 64;  // 32-column O blocks per warp (half of O's D columns)
+  const uint32_t bars = smem_u32(sm) + L::BAR_OFF;
+  const PrefillReq R = P.preq[pr.req];
+  const int warp = tid >> 5, lane = tid & 31;
+  const int qr = warp & 3, h = warp >> 2;
+  const int row = qr * 32 + lane;
+  const uint32_t lane_base = (uint32_t)(qr * 32) << 16;
+  const int pair_bar = 4 + qr;  // named barrier of warps qr and qr + 4
+  volatile float* xs = reinterpret_cast<volatile float*>(sm + L::XCH_OFF + row * L::XCH_STRIDE);
+  int lim[2], mask_from[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    lim[i] = R.prior + pr.qtile[i] * kQTile + row;  // last visible key of this row
+    mask_from[i] = R.prior + pr.qtile[i] * kQTile;
+  }
+  const float sc = P.scale_log2;
+  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+  bool failed = false;  // warp-uniform; after a failure only the barrier points are kept
+
+  for (int j = 0; j < pr.n; ++j) {
+    const uint32_t it = ps.kv + j;
+    const int tile0 = (pr.t0 + j) * kKVTile;
+    const int key_lo = tile0 + 64 * h;  // this warp's first key
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      if (!failed && !wait_bar_warp(bars + (L::B_SF + i) * 8, it & 1, P, abort_flag)) failed = true;
+      const uint32_t s_col = tmem + lane_base + 256 + 128 * i;
+      float s[64];
+      float mx = -INFINITY;
+      if (!failed) {
+        tc_fence_after();
+        {
+          uint32_t r0[32], r1[32];
+          tmem_ld32x2(s_col + 64 * h, r0, r1);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            s[c] = __uint_as_float(r0[c]);
+            s[32 + c] = __uint_as_float(r1[c]);
+          }
+        }
+        if (tile0 + kKVTile - 1 > mask_from[i]) {  // uniform over the warp pair
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (key_lo + c > lim[i]) s[c] = -INFINITY;
+        }
+        // 64 -> 22 -> 8 -> 3 -> 1 with three-input max
+        float a[22];
+#pragma unroll
+        for (int c = 0; c < 21; ++c) a[c] = max3(s[3 * c], s[3 * c + 1], s[3 * c + 2]);
+        a[21] = s[63];
+        float b[8];
+#pragma unroll
+        for (int c = 0; c < 7; ++c) b[c] = max3(a[3 * c], a[3 * c + 1], a[3 * c + 2]);
+        b[7] = a[21];
+        mx = max3(max3(b[0], b[1], b[2]), max3(b[3], b[4], b[5]), fmaxf(b[6], b[7]));
+        mx *= sc;
+      }
+      xs[2 * i + h] = mx;
+      asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
+      mx = fmaxf(mx, xs[2 * i + (h ^ 1)]);
+      if (!failed) {
+        // Lazy rescaling, as in the one-warp-per-row form: both warps of the
+        // pair compute the same reference from the same row max.
+        float alpha = 1.f;
+        bool rescale = false;
+        if (mx > m_run[i] + 8.f) {
+          alpha = ex2(m_run[i] - mx);
+          rescale = (m_run[i] != -INFINITY);
+          m_run[i] = mx;
+        }
+        const float m_use = (m_run[i] == -INFINITY) ? 0.f : m_run[i];
+        const uint64_t sc2 = f2_pack(sc, sc), nm2 = f2_pack(-m_use, -m_use);
+        uint64_t acc[4];
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          float x0, x1;
+          f2_unpack(ffma2(f2_pack(s[2 * c], s[2 * c + 1]), sc2, nm2), x0, x1);
+          const float p0 = ex2(x0), p1 = ex2(x1);
+          pk[c] = POD_PACK(p0, p1);
+          const uint64_t p2 = f2_pack(p0, p1);
+          acc[c & 3] = (c < 4) ? p2 : fadd2(acc[c & 3], p2);
+        }
+        tmem_st32(s_col + 32 * h, pk);
+        float a0, a1;
+        f2_unpack(fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3])), a0, a1);
+        l_run[i] = l_run[i] * alpha + (a0 + a1);
+        // O_i is stable here (S_i of this tile was issued after the previous
+        // PV_i completed); each warp rescales its half of O's columns.
+        if (__any_sync(0xffffffffu, rescale)) {
+          const float f = rescale ? alpha : 1.f;
+          const uint32_t o_col = tmem + lane_base + 128 * i + (D / 2) * h;
+#pragma unroll
+          for (int cb = 0; cb < OB; ++cb) {
+            uint32_t ov[32];
+            tmem_ld32(o_col + cb * 32, ov);
+#pragma unroll
+            for (int q = 0; q < 32; ++q) ov[q] = __float_as_uint(__uint_as_float(ov[q]) * f);
+            tmem_st32(o_col + cb * 32, ov);
+          }
+        }
+      }
+      // one arrival per warp, stores complete (tcgen05.wait::st) or none made
+      tc_fence_before();
+      __syncwarp();
+      if (!failed && lane == 0) mbar_arrive(bars + (L::B_PF + i) * 8);
+    }
+  }
+  // O_0 and O_1 complete
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    if (!failed) {
+      if (wait_bar_warp(bars + (L::B_OR + i) * 8, ps.units & 1, P, abort_flag))
+        tc_fence_after();
+      else
+        failed = true;
+    }
+  }
+  ps.kv += pr.n;
+  ps.units++;
+  // The two halves' row sums. The first barrier keeps this write behind the
+  // partner's last read of the max slots.
+  asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
+  xs[h] = l_run[0];
+  xs[2 + h] = l_run[1];
+  asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
+  const float l_tot[2] = {l_run[0] + xs[h ^ 1], l_run[1] + xs[2 + (h ^ 1)]};
+
+  if (pr.n_split <= 1) {
+    if (failed) return false;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const bool tile_ok = (i == 0) || pr.valid1;
+      const int q_local = pr.qtile[i] * kQTile + row;
+      const bool valid = tile_ok && (q_local < R.chunk);
+      const size_t out_row = (size_t)(R.q_row0 + q_local);
+      const float inv = 1.f / l_tot[i];
+      const uint32_t o_col = tmem + lane_base + 128 * i + (D / 2) * h;
+#pragma unroll
+      for (int cb = 0; cb < OB; ++cb) {
+        uint32_t ov[32];
+        tmem_ld32(o_col + cb * 32, ov);
+        if (valid) {
+          uint16_t* dst = P.o_p + (out_row * P.H + pr.head[i]) * D + (D / 2) * h + cb * 32;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 v;
+            v.x = pack_bf16(__uint_as_float(ov[8 * q + 0]) * inv, __uint_as_float(ov[8 * q + 1]) * inv);
+            v.y = pack_bf16(__uint_as_float(ov[8 * q + 2]) * inv, __uint_as_float(ov[8 * q + 3]) * inv);
+            v.z = pack_bf16(__uint_as_float(ov[8 * q + 4]) * inv, __uint_as_float(ov[8 * q + 5]) * inv);
+            v.w = pack_bf16(__uint_as_float(ov[8 * q + 6]) * inv, __uint_as_float(ov[8 * q + 7]) * inv);
+            *reinterpret_cast<uint4*>(dst + 8 * q) = v;
+          }
+        }
+      }
+      if (valid && h == 0) {
+        const float lse2 = (l_tot[i] > 0.f) ? (m_run[i] + log2f(l_tot[i])) : -INFINITY;
+        P.lse_p[out_row * P.H + pr.head[i]] = lse2 * kLn2;
+      }
+    }
+    return true;
+  }
+  // Split partials of both tiles: O normalised by its own sum (fp32), stored
+  // [slot][d / 4][row] in float4 units, and the natural-log LSE of the range.
+  float4* part = reinterpret_cast<float4*>(P.ppart_o);
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const bool tile_ok = (i == 0) || pr.valid1;
+    const bool valid = tile_ok && (pr.qtile[i] * kQTile + row < R.chunk) && !failed;
+    const int slot0 = pr.slot_base[i];
+    const float inv = (l_tot[i] > 0.f) ? 1.f / l_tot[i] : 0.f;
+    float4* po = part + (size_t)(slot0 + pr.split) * (D / 4) * kQTile + row;
+    const uint32_t o_col = tmem + lane_base + 128 * i + (D / 2) * h;
+#pragma unroll
+    for (int cb = 0; cb < OB && !failed; ++cb) {
+      uint32_t ov[32];
+      tmem_ld32(o_col + cb * 32, ov);
+      if (valid) {
+        const int c4 = (D / 8) * h + cb * 8;  // first float4 column of this block
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          po[(size_t)(c4 + q) * kQTile] =
+              make_float4(__uint_as_float(ov[4 * q]) * inv, __uint_as_float(ov[4 * q + 1]) * inv,
+                          __uint_as_float(ov[4 * q + 2]) * inv, __uint_as_float(ov[4 * q + 3]) * inv);
+      }
+    }
+    if (valid && h == 0) {
+      const float lse2 = (l_tot[i] > 0.f) ? (m_run[i] + log2f(l_tot[i])) : -INFINITY;
+      P.ppart_lse[(size_t)(slot0 + pr.split) * kQTile + row] = lse2 * kLn2;
+    }
+  }
+  // Both tiles' partials are written by all eight warps: one barrier of the
+  // eight, then one thread per tile counts the split in.
+  __threadfence();
+  asm volatile("bar.sync 2, %0;" ::"n"(kSoftmaxWarps * 32) : "memory");
+  if ((tid & 127) == 0) {
+    const int ti = tid >> 7;  // thread 0: tile 0, thread 128: tile 1
+    const bool ok_t = (ti == 0) || pr.valid1;
+    const int old = (*abort_flag || !ok_t) ? -1 : atomicAdd(P.pgroup_ctr + pr.group[ti], 1);
+    s_flag[ti] = (old == pr.n_split - 1);
+  }
+  asm volatile("bar.sync 2, %0;" ::"n"(kSoftmaxWarps * 32) : "memory");
+  // The last split to finish merges: warps 0-3 tile 0, warps 4-7 tile 1, one
+  // query row per thread, in split order (the result does not depend on which
+  // split finished last).
+  const int im = h;
+  const bool tile_ok_m = (im == 0) || pr.valid1;
+  const int q_local_m = pr.qtile[im] * kQTile + row;
+  if (s_flag[im] && !failed && tile_ok_m && q_local_m < R.chunk) {
+    __threadfence();
+    const size_t out_row = (size_t)(R.q_row0 + q_local_m);
+    const int slot0 = pr.slot_base[im];
+    const int ns = pr.n_split;
+    const float* pl = P.ppart_lse + (size_t)slot0 * kQTile + row;
+    float m = -INFINITY;
+    for (int sp = 0; sp < ns; ++sp) m = fmaxf(m, __ldcg(pl + (size_t)sp * kQTile));
+    float wsum = 0.f;
+    for (int sp = 0; sp < ns; ++sp) {
+      const float v = __ldcg(pl + (size_t)sp * kQTile);
+      wsum += (v == -INFINITY) ? 0.f : ex2((v - m) * kLog2e);
+    }
+    const float winv = 1.f / wsum;
+    uint16_t* dst = P.o_p + (out_row * P.H + pr.head[im]) * D;
+    const float4* src = part + (size_t)slot0 * (D / 4) * kQTile + row;
+#pragma unroll 1
+    for (int cb = 0; cb < D / 32; ++cb) {
+      float acc[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) acc[c] = 0.f;
+#pragma unroll 2
+      for (int sp = 0; sp < ns; ++sp) {
+        const float v = __ldcg(pl + (size_t)sp * kQTile);
+        const float w = ((v == -INFINITY) ? 0.f : ex2((v - m) * kLog2e)) * winv;
+        const float4* s4 = src + (size_t)sp * (D / 4) * kQTile + (size_t)(cb * 8) * kQTile;
+        float4 x[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) x[q] = __ldcg(s4 + (size_t)q * kQTile);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          acc[4 * q] = fmaf(w, x[q].x, acc[4 * q]);
+          acc[4 * q + 1] = fmaf(w, x[q].y, acc[4 * q + 1]);
+          acc[4 * q + 2] = fmaf(w, x[q].z, acc[4 * q + 2]);
+          acc[4 * q + 3] = fmaf(w, x[q].w, acc[4 * q + 3]);
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint4 v;
+        v.x = pack_bf16(acc[8 * q + 0], acc[8 * q + 1]);
+        v.y = pack_bf16(acc[8 * q + 2], acc[8 * q + 3]);
+        v.z = pack_bf16(acc[8 * q + 4], acc[8 * q + 5]);
+        v.w = pack_bf16(acc[8 * q + 6], acc[8 * q + 7]);
+        *reinterpret_cast<uint4*>(dst + cb * 32 + 8 * q) = v;
+      }
+    }
+    P.lse_p[out_row * P.H + pr.head[im]] = m + logf(wsum);
+  }
+  return !failed;
+}
+
 // ---- softmax + epilogue: warps 0-3 serve query tile 0, warps 4-7 tile 1; one
 // thread per query row (TMEM lane), 128 keys per S tile in two 64-column halves.
 template <int D>
