@@ -123,10 +123,11 @@ class ClockSampler:
             except Exception:
                 self.proc.kill()
 
-    def summary(self):
-        sm, mx, reasons = [], [], set()
+    def summary(self, lo=0, hi=None):
+        """Median SM clock (and power) over samples lo..hi, with every throttle reason seen."""
+        sm, mx, pw, reasons = [], [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for ln in self.lines[lo:hi]:
             parts = [x.strip() for x in ln.split(",")]
             if len(parts) < 8:
                 continue
@@ -135,13 +136,20 @@ class ClockSampler:
                 mx.append(float(parts[1]))
             except ValueError:
                 continue
+            try:
+                pw.append(float(parts[2]))
+            except ValueError:
+                pass
             for name, v in zip(names, parts[4:8]):
                 if v.lower().startswith("active"):
                     reasons.add(name)
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
-                "reasons": sorted(reasons)}
+        out = {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+               "reasons": sorted(reasons)}
+        if pw:
+            out["power_w"] = statistics.median(pw)
+        return out
 
 
 def dist_setup(n_gpus):
@@ -234,6 +242,38 @@ def time_calls(fn, n, flush_buf, stream):
         times.append((s, e))
     torch.cuda.synchronize()
     return [s.elapsed_time(e) * 1000.0 for s, e in times]  # us
+
+
+def sustained(fn, seconds, stream, local):
+    """Back-to-back calls (no L2 flush) for `seconds` after one second of the same
+    load, so the board's power limit has settled: mean us per call and the SM
+    clock and power sampled over the timed part."""
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t0 = time.perf_counter()
+        while time.perf_counter() - t0 < 1.0:  # settle: same load, not timed
+            for _ in range(10):
+                fn()
+            torch.cuda.synchronize()
+        lo = len(clk.lines)
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        n = 0
+        s.record(stream)
+        t1 = time.perf_counter()
+        while time.perf_counter() - t1 < seconds:
+            for _ in range(20):
+                fn()
+            n += 20
+            torch.cuda.synchronize()
+        e.record(stream)
+        torch.cuda.synchronize()
+        hi = len(clk.lines)
+    out = {"us_per_call": s.elapsed_time(e) * 1000.0 / n, "calls": n}
+    out.update(clk.summary(lo, hi))
+    return out
 
 
 def mean(xs):
@@ -351,6 +391,24 @@ def run_gpu(args, rank, world, local):
     two = time_calls(call(pa.MODE_TWO_STREAM), extra_steps, flush, stream)
     p_only = time_calls(lambda: pod.prefill_only(pre, stream), extra_steps, flush, stream) if pre else [0.0]
     d_only = time_calls(lambda: pod.decode_only(dec, stream), extra_steps, flush, stream) if dec else [0.0]
+    # ---- sustained: each mode back to back under the board's power limit
+    sus = None
+    if world == 1 and args.sustained_seconds > 0:
+        sus = {"note": "calls back to back without L2 flush, after 1 s of the same load; "
+                       "clock and power are nvidia-smi medians over the timed part"}
+        modes = [("fused", call(pa.MODE_FUSED)), ("serial", call(pa.MODE_SERIAL)),
+                 ("two_stream", call(pa.MODE_TWO_STREAM))]
+        if pre:
+            modes.append(("prefill_only", lambda: pod.prefill_only(pre, stream)))
+        if dec:
+            modes.append(("decode_only", lambda: pod.decode_only(dec, stream)))
+        for name, fn in modes:
+            sus[name] = sustained(fn, args.sustained_seconds, stream, local)
+        # a step timed inside a long loop takes the sustained tensor peak
+        sus_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+        t_sus = max(F / (sus_peak * 1e12), B / (peaks["hbm_gbs"] * 1e9)) * 1e6
+        sus["fused"]["roofline_frac_sustained_peak"] = t_sus / sus["fused"]["us_per_call"]
+        sus["sustained_tensor_peak_tflops"] = sus_peak
     pod.hybrid(pre, dec, pa.MODE_FUSED, stream)
     plan = pod.last_plan()
     stats = pod.stats(stream) if args.stats else None
@@ -419,6 +477,7 @@ def run_gpu(args, rank, world, local):
         "plan": plan,
         "other_workloads": extras,
         "clocks": clocks,
+        "sustained": sus,
         "gpu_launches": args.steps,
         "wall_s_timed_region": wall,
         "cpu_baseline": cpu,
@@ -569,6 +628,8 @@ def main():
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the other full-size configurations")
     ap.add_argument("--extra-steps", type=int, default=10)
+    ap.add_argument("--sustained-seconds", type=float, default=2.0,
+                    help="per mode, back-to-back timing under the power limit (0: skip)")
     ap.add_argument("--stats", action="store_true")
     ap.add_argument("--sweep", default=None, choices=["chunked16k", "policies"],
                     help="ablation sweeps: the chunked 16K prompt (split limit, prefill tile) "
