@@ -59,6 +59,19 @@ constexpr int kSoftPairs = POD_SOFT_EXP2_PAIRS;
 #ifndef POD_SOFTMAX_SPLIT
 #define POD_SOFTMAX_SPLIT 0
 #endif
+// TMEM use of the one-SM prefill tile. 1 (default): one S buffer that the two
+// query tiles take in turn and a separate P_i per tile, so the next S is
+// issued as soon as the softmax has loaded the last one. 0: S_i per query
+// tile, P_i written over S_i (the next S_i waits for P_i V to complete).
+// Measured on B200, long-context batch (64 / 8 heads, d 128): the shared S
+// takes about 13 % fewer SM cycles per KV step, but the board's power limit
+// lowers the clock with it, so the call is 1-2 % faster.
+#ifndef POD_SHARED_S
+#define POD_SHARED_S 1
+#endif
+#if POD_SHARED_S && POD_SOFTMAX_SPLIT
+#error "the key-split softmax writes P over S_i: it needs POD_SHARED_S=0"
+#endif
 
 // L2 cache-policy hints: the decode K/V copies are evict-first (read once), so
 // the decode stream of a fused launch does not push the prefill's K/V tiles
@@ -137,9 +150,11 @@ struct FusedLayout {
   static constexpr int B_VF = B_KE + kPrefillStages;    // V tile landed
   static constexpr int B_VE = B_VF + kPrefillStages;    // V tile read by both PV MMAs
   static constexpr int B_SF = B_VE + kPrefillStages;    // S_i in TMEM [2]
-  static constexpr int B_SE = B_SF + 2;                 // S_i free (its P read by PV_i) [2]
+  static constexpr int B_SE = B_SF + 2;                 // S_i free (its P read by PV_i) [2];
+                                                        // shared S: [0] the S buffer loaded
   static constexpr int B_PF = B_SE + 2;                 // P_i in TMEM, one arrival per warp [2]
-  static constexpr int B_OR = B_PF + 2;                 // O_i final for the unit [2]
+  static constexpr int B_PE = B_PF + 2;                 // shared S: P_i read by PV_i [2]
+  static constexpr int B_OR = B_PE + 2;                 // O_i final for the unit [2]
   static constexpr int N_BARS = B_OR + 2;
   static constexpr int MISC_OFF = BAR_OFF + N_BARS * 8;
   static constexpr int TOTAL = MISC_OFF + 64;
@@ -609,6 +624,8 @@ __global__ void __launch_bounds__(kFusedThreads, kFusedSlotsPerSm)
       uint32_t cnt = 1;
       if (i == L::B_PF || i == L::B_PF + 1)  // one arrival per softmax warp of the tile
         cnt = POD_SOFTMAX_SPLIT ? kSoftmaxWarps : kSoftmaxWarps / 2;
+      if (POD_SHARED_S && i == L::B_SE)  // one arrival per warp of the tile that loaded S
+        cnt = kSoftmaxWarps / 2;
       mbar_init(bars + i * 8, cnt);
     }
     fence_mbar_init();

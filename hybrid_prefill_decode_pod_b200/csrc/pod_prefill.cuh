@@ -11,10 +11,15 @@
 //   warps 0-3   softmax of tile 0, warps 4-7 softmax of tile 1: one thread per
 //               query row (= TMEM lane), 128 keys per KV tile.
 // (Warps 10-11 of the CTA stream decode units meanwhile; see pod_kernels.cu.)
-// TMEM (512 columns): O0 [0,128), O1 [128,256), S0 [256,384), S1 [384,512);
-// P_i (bf16 pairs) is written over the first 64 columns of S_i.
-// MMA order S0 S1 | PV0 S0' | PV1 S1' | ...: while one softmax group works on
-// its tile the tensor core runs the other group's MMAs (ping-pong).
+// TMEM (512 columns), default layout: O0 [0,128), O1 [128,256), one S buffer
+// [256,384) that the two tiles take in turn, P0 [384,448), P1 [448,512) (bf16
+// pairs). A softmax warp frees the S buffer as soon as it has loaded its row,
+// so the next S is issued while it computes; MMA order S0 S1 | S0' PV0 |
+// S1' PV1 | ... The softmax waits for the previous P_i V before it rewrites
+// P_i (and rescales O_i).
+// With POD_SHARED_S=0: S0 [256,384), S1 [384,512), P_i written over the first
+// 64 columns of S_i, and S_i' waits for P_i V to complete (order S0 S1 | PV0
+// S0' | PV1 S1').
 // This is the FlashAttention-style tile of the POD-Attention summary (§1,
 // §A.1) rebuilt for Blackwell; the pairing plays the role of the paper's
 // larger prefill tile when fewer CTAs share an SM (§4.2.2).
@@ -179,8 +184,16 @@ POD_DEV bool prefill_mma(const Plan& P, const PrefillRange& pr, uint8_t* sm, uin
     const uint32_t it = ps.kv + j;
     const uint32_t st = it % kPrefillStages, ph = (it / kPrefillStages) & 1;
     if (i == 0 && !wait_bar(bars + (L::B_KF + st) * 8, ph, P, abort_flag)) return false;
+#if POD_SHARED_S
+    // the S buffer's previous content (use m - 1) has been loaded by its softmax
+    const uint32_t m = 2 * it + (uint32_t)i;
+    if (m >= 1 && !wait_bar(bars + L::B_SE * 8, (m - 1) & 1, P, abort_flag)) return false;
+    const uint32_t s_tm = tmem + 256;
+#else
     // S_i still holds P_i of the previous tile until that PV has read it
     if (it >= 1 && !wait_bar(bars + (L::B_SE + i) * 8, (it - 1) & 1, P, abort_flag)) return false;
+    const uint32_t s_tm = tmem + 256 + 128 * i;
+#endif
     tc_fence_after();
     const uint64_t qd = i ? dq1 : dq0;
     const uint64_t kd = dk0 + st * kStageStep;
@@ -188,7 +201,7 @@ POD_DEV bool prefill_mma(const Plan& P, const PrefillRange& pr, uint8_t* sm, uin
     for (int kk = 0; kk < KS; ++kk) {
       const uint64_t ad = qd + (uint64_t)(((kk >> 2) * (kQTile * 128) + (kk & 3) * 32) >> 4);
       const uint64_t bd = kd + (uint64_t)(((kk >> 2) * (kKVTile * 128) + (kk & 3) * 32) >> 4);
-      umma_ss(tmem + 256 + 128 * i, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
+      umma_ss(s_tm, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
     }
     umma_commit(bars + (L::B_SF + i) * 8);
     if (i == 1) umma_commit(bars + (L::B_KE + st) * 8);  // both S have read K_j
@@ -204,26 +217,36 @@ POD_DEV bool prefill_mma(const Plan& P, const PrefillRange& pr, uint8_t* sm, uin
     if (!wait_bar(bars + (L::B_PF + i) * 8, it & 1, P, abort_flag)) return false;
     tc_fence_after();
     const uint64_t vd = dv0 + st * kStageStep;
-    const uint32_t pcol = tmem + 256 + 128 * i;
+    const uint32_t pcol = tmem + (POD_SHARED_S ? 384 + 64 * i : 256 + 128 * i);
 #pragma unroll
     for (int kk = 0; kk < kKVTile / 16; ++kk) {
       const uint64_t bd = vd + (uint64_t)((kk * 16 * 128) >> 4);
       umma_ts(tmem + 128 * i, pcol + kk * 8, bd, IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
     }
-    umma_commit(bars + (L::B_SE + i) * 8);  // S_i free again
+    // P_i read (shared S: P_i may be rewritten; else S_i is free again)
+    const uint32_t done_bar = bars + ((POD_SHARED_S ? L::B_PE : L::B_SE) + i) * 8;
+    umma_commit(done_bar);
     if (j == pr.n - 1) umma_commit(bars + (L::B_OR + i) * 8);  // O_i final for this unit
     if (i == 1) umma_commit(bars + (L::B_VE + st) * 8);      // both PV have read V_j
-    last_commit_bar = bars + (L::B_SE + i) * 8;
+    last_commit_bar = done_bar;
     last_commit_par = it & 1;
     return true;
   };
 
   if (!issue_s(0, 0) || !issue_s(1, 0)) return false;
   for (int j = 0; j < pr.n; ++j) {
+#if POD_SHARED_S
+    // S0' as soon as the buffer is free, while the softmax of tile 0 still works
+    if (j + 1 < pr.n && !issue_s(0, j + 1)) return false;
+    if (!issue_pv(0, j)) return false;
+    if (j + 1 < pr.n && !issue_s(1, j + 1)) return false;
+    if (!issue_pv(1, j)) return false;
+#else
     if (!issue_pv(0, j)) return false;
     if (j + 1 < pr.n && !issue_s(0, j + 1)) return false;
     if (!issue_pv(1, j)) return false;
     if (j + 1 < pr.n && !issue_s(1, j + 1)) return false;
+#endif
   }
   ps.kv += pr.n;
   return true;
@@ -519,7 +542,8 @@ POD_DEV bool prefill_softmax(const Plan& P, const PrefillRange& pr, uint8_t* sm,
   const int i = warp >> 2;  // which query tile of the unit
   const int row = (warp & 3) * 32 + lane;
   const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-  const uint32_t s_col = tmem + lane_base + 256 + 128 * i;
+  const uint32_t s_col = tmem + lane_base + (POD_SHARED_S ? 256 : 256 + 128 * i);
+  const uint32_t p_col = tmem + lane_base + (POD_SHARED_S ? 384 + 64 * i : 256 + 128 * i);
   const uint32_t o_col = tmem + lane_base + 128 * i;
   const int head = pr.head[i], qtile = pr.qtile[i];
   const bool tile_ok = (i == 0) || pr.valid1;  // uniform over the warp group
@@ -547,6 +571,12 @@ POD_DEV bool prefill_softmax(const Plan& P, const PrefillRange& pr, uint8_t* sm,
 #pragma unroll
       for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(r[c]);
     }
+#if POD_SHARED_S
+    // S is in registers (the load waited): the buffer may take the next S
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bars + L::B_SE * 8);
+#endif
     if (masked_tile) {
 #pragma unroll
       for (int c = 0; c < 128; ++c)
@@ -579,8 +609,9 @@ POD_DEV bool prefill_softmax(const Plan& P, const PrefillRange& pr, uint8_t* sm,
     // x = s sc - m and the row sums on packed pairs (f32x2)
     const uint64_t sc2 = f2_pack(sc, sc), nm2 = f2_pack(-m_use, -m_use);
     uint64_t acc[4];
-    // P (bf16 pairs) over S columns 0..63, already read; the PV MMA reads it
-    // as A. Keys 64 hh .. +63 go to columns 32 hh .. +31.
+    // P (bf16 pairs) in 64 columns (over S_i's first 64, already read, or in
+    // P_i's own columns with a shared S buffer); the PV MMA reads it as A.
+    // Keys 64 hh .. +63 go to columns 32 hh .. +31.
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
       uint32_t pk[32];
@@ -604,11 +635,22 @@ POD_DEV bool prefill_softmax(const Plan& P, const PrefillRange& pr, uint8_t* sm,
         // unrounded weights (see the decode path), four running pair sums
         acc[c & 3] = (hh == 0 && c < 4) ? p2 : fadd2(acc[c & 3], p2);
       }
+#if POD_SHARED_S
+      if (hh == 0 && it >= 1) {
+        // P_i (and O_i, rescaled below) are still read by the previous P_i V
+        if (!wait_bar_warp(bars + (L::B_PE + i) * 8, (it - 1) & 1, P, abort_flag)) {
+          failed = true;
+          break;
+        }
+        tc_fence_after();
+      }
+#endif
       if (hh == 0)
-        tmem_st32_nowait(s_col, pk);
+        tmem_st32_nowait(p_col, pk);
       else
-        tmem_st32(s_col + 32, pk);  // waits for both stores
+        tmem_st32(p_col + 32, pk);  // waits for both stores
     }
+    if (failed) break;
     float lt;
     {
       float a0, a1;
@@ -616,8 +658,9 @@ POD_DEV bool prefill_softmax(const Plan& P, const PrefillRange& pr, uint8_t* sm,
       lt = a0 + a1;
     }
     l_run = l_run * alpha + lt;
-    // O_i is stable here: S_i of this tile was issued only after the previous
-    // PV_i completed. tcgen05.ld/st are warp-collective, so the whole warp
+    // O_i is stable here: the previous PV_i has completed (S_i of this tile was
+    // issued only after it, or with a shared S buffer the wait before the P
+    // store saw it). tcgen05.ld/st are warp-collective, so the whole warp
     // takes this branch if any row rescales; the others multiply by 1.
     if (__any_sync(0xffffffffu, rescale)) {
       const float f = rescale ? alpha : 1.f;
