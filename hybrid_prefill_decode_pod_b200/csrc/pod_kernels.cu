@@ -69,9 +69,6 @@ constexpr int kSoftPairs = POD_SOFT_EXP2_PAIRS;
 #ifndef POD_SHARED_S
 #define POD_SHARED_S 1
 #endif
-#if POD_SHARED_S && POD_SOFTMAX_SPLIT
-#error "the key-split softmax writes P over S_i: it needs POD_SHARED_S=0"
-#endif
 
 // L2 cache-policy hints: the decode K/V copies are evict-first (read once), so
 // the decode stream of a fused launch does not push the prefill's K/V tiles
@@ -624,8 +621,8 @@ __global__ void __launch_bounds__(kFusedThreads, kFusedSlotsPerSm)
       uint32_t cnt = 1;
       if (i == L::B_PF || i == L::B_PF + 1)  // one arrival per softmax warp of the tile
         cnt = POD_SOFTMAX_SPLIT ? kSoftmaxWarps : kSoftmaxWarps / 2;
-      if (POD_SHARED_S && i == L::B_SE)  // one arrival per warp of the tile that loaded S
-        cnt = kSoftmaxWarps / 2;
+      if (POD_SHARED_S && i == L::B_SE)  // one arrival per warp that loads a part of S
+        cnt = POD_SOFTMAX_SPLIT ? kSoftmaxWarps : kSoftmaxWarps / 2;
       mbar_init(bars + i * 8, cnt);
     }
     fence_mbar_init();

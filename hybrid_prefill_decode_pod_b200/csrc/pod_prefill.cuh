@@ -263,8 +263,9 @@ POD_DEV bool prefill_mma(const Plan& P, const PrefillRange& pr, uint8_t* sm, uin
 //     the same row max, reference max and rescale decision;
 //   - at the end of the unit, the two partial row sums.
 // Each warp writes the P columns of its own keys (P of keys 64 h .. +63 goes to
-// S columns 32 h .. +31; the pair barrier orders that store after the other
-// warp's S load) and rescales and stores its half of O's columns.
+// P columns 32 h .. +31: P_i's own columns with the shared S buffer, else S_i's,
+// where the pair barrier orders that store after the other warp's S load) and
+// rescales and stores its half of O's columns.
 template <int D>
 POD_DEV bool prefill_softmax_split(const Plan& P, const PrefillRange& pr, uint8_t* sm,
                                    uint32_t tmem, PipeState& ps, int tid,
@@ -296,7 +297,8 @@ POD_DEV bool prefill_softmax_split(const Plan& P, const PrefillRange& pr, uint8_
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
       if (!failed && !wait_bar_warp(bars + (L::B_SF + i) * 8, it & 1, P, abort_flag)) failed = true;
-      const uint32_t s_col = tmem + lane_base + 256 + 128 * i;
+      const uint32_t s_col = tmem + lane_base + (POD_SHARED_S ? 256 : 256 + 128 * i);
+      const uint32_t p_col = tmem + lane_base + (POD_SHARED_S ? 384 + 64 * i : 256 + 128 * i);
       float s[64];
       float mx = -INFINITY;
       if (!failed) {
@@ -310,6 +312,13 @@ POD_DEV bool prefill_softmax_split(const Plan& P, const PrefillRange& pr, uint8_
             s[32 + c] = __uint_as_float(r1[c]);
           }
         }
+#if POD_SHARED_S
+        // this warp's half of S is in registers; the buffer takes the next S
+        // once all eight warps have loaded theirs
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars + L::B_SE * 8);
+#endif
         if (tile0 + kKVTile - 1 > mask_from[i]) {  // uniform over the warp pair
 #pragma unroll
           for (int c = 0; c < 64; ++c)
@@ -353,13 +362,24 @@ POD_DEV bool prefill_softmax_split(const Plan& P, const PrefillRange& pr, uint8_
           const uint64_t p2 = f2_pack(p0, p1);
           acc[c & 3] = (c < 4) ? p2 : fadd2(acc[c & 3], p2);
         }
-        tmem_st32(s_col + 32 * h, pk);
+#if POD_SHARED_S
+        // P_i (and O_i, rescaled below) are still read by the previous P_i V
+        if (it >= 1) {
+          if (wait_bar_warp(bars + (L::B_PE + i) * 8, (it - 1) & 1, P, abort_flag))
+            tc_fence_after();
+          else
+            failed = true;
+        }
+        if (!failed) tmem_st32(p_col + 32 * h, pk);
+#else
+        tmem_st32(p_col + 32 * h, pk);
+#endif
         float a0, a1;
         f2_unpack(fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3])), a0, a1);
         l_run[i] = l_run[i] * alpha + (a0 + a1);
         // O_i is stable here (S_i of this tile was issued after the previous
         // PV_i completed); each warp rescales its half of O's columns.
-        if (__any_sync(0xffffffffu, rescale)) {
+        if (!failed && __any_sync(0xffffffffu, rescale)) {
           const float f = rescale ? alpha : 1.f;
           const uint32_t o_col = tmem + lane_base + 128 * i + (D / 2) * h;
 #pragma unroll
