@@ -80,3 +80,27 @@ def test_reference_arm_under_torchrun_prints_one_line_from_rank0():
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
     # full oracle calls, the steps that ran reported as such
     assert d["steps"] == 2 and d["warmup"] == 0 and "unsampled" in d["cpu_baseline"]["sample"]
+
+
+def test_clock_summary_reads_medians_power_and_throttle_reasons():
+    # nvidia-smi csv,noheader,nounits lines in ClockSampler.FIELDS order:
+    # clocks.sm, clocks.max.sm, power.draw, reasons.active, hw_slowdown,
+    # hw_thermal_slowdown, sw_thermal_slowdown, sw_power_cap
+    sys.path.insert(0, ROOT)
+    import bench
+    c = bench.ClockSampler(0)
+    c.lines = [
+        "1965, 1965, 250.0, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "1530, 1965, 990.5, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "1540, 1965, 991.5, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "1550, 1965, 992.5, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "garbage line",
+    ]
+    s = bench.ClockSampler.summary(c)
+    assert s["sm_mhz"] == 1545.0 and s["sm_max_mhz"] == 1965.0 and s["samples"] == 4
+    assert s["reasons"] == ["sw_power_cap"]
+    # a window of the samples (the sustained timing skips its settling second)
+    w = c.summary(1, 4)
+    assert w["sm_mhz"] == 1540.0 and w["power_w"] == 991.5 and w["samples"] == 3
+    c.lines = []
+    assert c.summary()["reasons"] == ["unavailable"]
