@@ -5,9 +5,10 @@
 //  * prefill unit (pod_prefill.cuh): two 128-row query tiles that share K/V
 //    against a range of 128-key KV tiles. A TMA producer warp stages Q and
 //    K/V (128-byte swizzle), one thread issues tcgen05.mma (S_i = Q_i K^T into
-//    TMEM, O_i += P_i V with P_i read from TMEM), and two groups of four
-//    softmax warps (one thread per query row = TMEM lane) run the online
-//    softmax of the two tiles in ping-pong with the tensor pipe.
+//    a TMEM S buffer the two tiles take in turn, O_i += P_i V with P_i read
+//    from its own TMEM columns), and two groups of four softmax warps (one
+//    thread per query row = TMEM lane) run the online softmax of the two
+//    tiles while the tensor pipe works on the other tile's MMAs.
 //  * decode unit: one warp (a "virtual decode CTA", paper §4.2.3) streams the
 //    K/V rows of (request, KV head, key split) with 16-byte cp.async copies
 //    into a padded smem ring and runs S^T = K Q^T and O^T += V^T P^T on the

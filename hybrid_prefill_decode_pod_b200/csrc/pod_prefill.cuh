@@ -156,7 +156,8 @@ POD_DEV void prefill_producer_drain(const Plan& P, uint8_t* sm, const PipeState&
   }
 }
 
-// ---- MMA issuer (one thread). TMEM columns: O_i at 128 i, S_i at 256 + 128 i.
+// ---- MMA issuer (one thread). TMEM columns: O_i at 128 i; the shared S buffer
+// at 256 and P_i at 384 + 64 i (with POD_SHARED_S=0: S_i and P_i at 256 + 128 i).
 template <int D>
 POD_DEV bool prefill_mma(const Plan& P, const PrefillRange& pr, uint8_t* sm, uint32_t tmem,
                          PipeState& ps, uint32_t& last_commit_bar, uint32_t& last_commit_par,
